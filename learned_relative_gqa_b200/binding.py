@@ -1,0 +1,194 @@
+"""Thin Python binding of ``libinkling_rel_attn.so``.
+
+Argument marshalling only: every step of the attention runs in the library's
+CUDA kernels. The functions carry the C entry points' names; tensors are
+PyTorch device tensors (PyTorch supplies device memory and streams), passed
+to the library as raw pointers. There is no fallback: if the library is
+missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libinkling_rel_attn.so")
+
+INKLING_OK = 0
+INKLING_ERR_INVALID_ARG = 1
+INKLING_ERR_UNSUPPORTED = 2
+INKLING_ERR_MALFORMED_POSITIONS = 3
+INKLING_ERR_TIMEOUT = 4
+INKLING_ERR_CUDA = 5
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "seq_q", "seq_k", "heads_q", "heads_kv", "head_dim", "rel_extent", "window", "query_offset")]
+
+
+class InklingError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if status == INKLING_ERR_CUDA:
+            msg += f": {load().inkling_rel_attn_last_cuda_error().decode()}"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{os.path.basename(path)} is not built; run python -m learned_relative_gqa_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    dp = ctypes.POINTER(Dims)
+    lib.inkling_rel_attn_workspace_size.restype = sz
+    lib.inkling_rel_attn_workspace_size.argtypes = [dp, ctypes.c_int]
+    lib.inkling_rel_attn_validate.restype = ctypes.c_int
+    lib.inkling_rel_attn_validate.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
+    lib.inkling_rel_attn_fwd.restype = ctypes.c_int
+    lib.inkling_rel_attn_fwd.argtypes = [dp] + [vp] * 11 + [vp, sz, vp]
+    lib.inkling_rel_attn_bwd.restype = ctypes.c_int
+    lib.inkling_rel_attn_bwd.argtypes = [dp] + [vp] * 18 + [vp, sz, vp]
+    lib.inkling_rel_attn_last_device_error.restype = ctypes.c_int
+    lib.inkling_rel_attn_last_device_error.argtypes = [vp, vp]
+    lib.inkling_rel_attn_selftest_wait_timeout.restype = ctypes.c_int
+    lib.inkling_rel_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
+    lib.inkling_rel_attn_set_timing_events.restype = ctypes.c_int
+    lib.inkling_rel_attn_set_timing_events.argtypes = [vp, ctypes.c_int]
+    lib.inkling_rel_attn_last_cuda_error.restype = ctypes.c_char_p
+    lib.inkling_rel_attn_last_cuda_error.argtypes = []
+    lib.inkling_status_string.restype = ctypes.c_char_p
+    lib.inkling_status_string.argtypes = [ctypes.c_int]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().inkling_status_string(int(status)).decode()
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_dims(q: torch.Tensor, k: torch.Tensor, profiles: Optional[torch.Tensor], window: int,
+              query_offset: int = 0, rel_extent: Optional[int] = None) -> Dims:
+    B, S, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    R = profiles.shape[3] if profiles is not None else int(rel_extent or 0)
+    return Dims(B, S, Skv, Hq, Hkv, D, R, int(window), int(query_offset))
+
+
+def inkling_rel_attn_workspace_size(dims: Dims, backward: bool) -> int:
+    return int(load().inkling_rel_attn_workspace_size(ctypes.byref(dims), int(bool(backward))))
+
+
+def alloc_workspace(dims: Dims, backward: bool, device) -> torch.Tensor:
+    n = inkling_rel_attn_workspace_size(dims, backward)
+    if n == 0:
+        raise InklingError(INKLING_ERR_INVALID_ARG, "workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _u8(t):
+    return None if t is None else (t if t.dtype == torch.uint8 else t.view(torch.uint8) if t.dtype == torch.bool
+                                   else t.to(torch.uint8))
+
+
+def _check(status: int, where: str):
+    if status != INKLING_OK:
+        raise InklingError(status, where)
+
+
+def inkling_rel_attn_validate(dims: Dims, valid, key_valid, positions, key_positions, workspace,
+                              stream=None) -> int:
+    """Returns the library status (INKLING_OK or INKLING_ERR_MALFORMED_POSITIONS, ...)."""
+    return int(load().inkling_rel_attn_validate(
+        ctypes.byref(dims), _p(_u8(valid)), _p(_u8(key_valid)), _p(positions), _p(key_positions),
+        _p(workspace), workspace.numel(), _stream(stream)))
+
+
+def inkling_rel_attn_fwd(dims: Dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions,
+                         out, lse, workspace, stream=None) -> None:
+    st = load().inkling_rel_attn_fwd(
+        ctypes.byref(dims), _p(q), _p(k), _p(v), _p(profiles), _p(sink), _p(_u8(valid)), _p(_u8(key_valid)),
+        _p(positions), _p(key_positions), _p(out), _p(lse), _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_rel_attn_fwd")
+
+
+def inkling_rel_attn_bwd(dims: Dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions,
+                         out, lse, dout, dlse, dq, dk, dv, dprofiles, dsink, workspace, stream=None) -> None:
+    st = load().inkling_rel_attn_bwd(
+        ctypes.byref(dims), _p(q), _p(k), _p(v), _p(profiles), _p(sink), _p(_u8(valid)), _p(_u8(key_valid)),
+        _p(positions), _p(key_positions), _p(out), _p(lse), _p(dout), _p(dlse), _p(dq), _p(dk), _p(dv),
+        _p(dprofiles), _p(dsink), _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_rel_attn_bwd")
+
+
+def inkling_rel_attn_last_device_error(workspace, stream=None) -> int:
+    return int(load().inkling_rel_attn_last_device_error(_p(workspace), _stream(stream)))
+
+
+def inkling_rel_attn_selftest_wait_timeout(timeout_us: int, workspace, stream=None) -> int:
+    return int(load().inkling_rel_attn_selftest_wait_timeout(int(timeout_us), _p(workspace), workspace.numel(),
+                                                             _stream(stream)))
+
+
+def inkling_rel_attn_set_timing_events(events, n_pairs: int) -> None:
+    """events: a ctypes array of cudaEvent_t handles (or None to switch the hook off)."""
+    _check(load().inkling_rel_attn_set_timing_events(events, int(n_pairs)), "inkling_rel_attn_set_timing_events")
+
+
+# --------------------------------------------------------------------------
+# convenience wrappers (allocate outputs with torch, then call the entry points)
+# --------------------------------------------------------------------------
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def forward(q, k, v, profiles, sink, valid, key_valid=None, positions=None, key_positions=None, *,
+            window: int = 0, query_offset: int = 0, workspace=None, stream=None):
+    """out [B,S,Hq,D] fp32 and lse [B,S,Hq] fp32 (see include/inkling_rel_attn.h)."""
+    _contig(q, k, v, profiles, sink, valid, key_valid, positions, key_positions)
+    dims = make_dims(q, k, profiles, window, query_offset)
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ws = alloc_workspace(dims, False, q.device) if workspace is None else workspace
+    inkling_rel_attn_fwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, ws,
+                         stream)
+    return out, lse
+
+
+def backward(q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout, dlse=None, *,
+             window: int = 0, query_offset: int = 0, workspace=None, stream=None):
+    """dict dq, dk, dv, dprofiles, dsink (fp32)."""
+    _contig(q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout, dlse)
+    dims = make_dims(q, k, profiles, window, query_offset)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(q.shape, **f32)
+    dk = torch.empty(k.shape, **f32)
+    dv = torch.empty(v.shape, **f32)
+    dprof = torch.empty(profiles.shape, **f32)
+    dsink = torch.empty(sink.shape, **f32)
+    ws = alloc_workspace(dims, True, q.device) if workspace is None else workspace
+    inkling_rel_attn_bwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout,
+                         dlse, dq, dk, dv, dprof, dsink, ws, stream)
+    return dict(dq=dq, dk=dk, dv=dv, dprofiles=dprof, dsink=dsink)

@@ -1,0 +1,752 @@
+// bwd.cu -- backward kernels of learned-relative grouped-query attention (sm_100a).
+//
+// The backward recomputes probabilities from the forward's log-sum-exp
+// (P = exp(z - lse), sink included in lse) and applies the softmax chain rule
+//   dP = dout . v,  dz = P (dP - Dv),  Dv = <dout, out> - dlse,
+//   dq = scale sum_j dz k_j,  dk = scale sum_i dz q_i,  dv = sum_i P dout_i,
+//   dprofiles[b,h,i,d] = dz for the allowed key at distance d < R.
+// Dv, dsink, a BF16 copy of dout and lse*log2(e) come from the preprocessing
+// kernel; dprofiles entries that no allowed key reaches are zeroed there too.
+//
+// Two kernels, both tensor-core (tcgen05) with TMEM accumulators:
+//   * dkdv: one CTA per (batch, KV head, 128-key tile). It walks every query
+//     head of the group and every 64-row query tile that sees the key tile,
+//     computing S^T = K Q^T and dP^T = V dO^T (keys on TMEM lanes), then
+//     dV += P^T dO and dK += dS^T Q with P^T / dS^T taken from TMEM. With keys
+//     on the lanes, the dprofiles row of a query is written by 32 consecutive
+//     distances per warp store (coalesced), with plain stores: each (i, d)
+//     has exactly one allowed key.
+//   * dq: one CTA per (batch, query head, 128-row query tile) over 64-key
+//     tiles: S = Q K^T, dP = dO V^T, dQ += dS K (dS from TMEM). No atomics.
+// In both, S/dP are double buffered in TMEM and two softmax warpgroups take
+// alternate steps, so the MMAs of one step overlap the other's elementwise work.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace ira {
+namespace bwdk {
+
+__device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
+__device__ __forceinline__ int ceil_div_i(int a, int b) { return -floor_div(-a, b); }
+
+// =====================================================================================
+// dK / dV / dprofiles
+// =====================================================================================
+namespace kv {
+
+constexpr int BK = 128;              // keys per CTA (TMEM lanes)
+constexpr int BQ = 64;               // queries per step
+constexpr int BAND_CHUNKS = 17;      // 16-B chunks per band row
+constexpr int BAND_PITCH = BAND_CHUNKS * 16;
+constexpr int BAND_BYTES = BQ * BAND_PITCH;
+constexpr int KTILE = BK * 128;      // [128 rows x 64 bf16] box
+constexpr int QTILE = BQ * 128;      // [64 rows x 64 bf16] box
+
+struct StepInfo {
+    int lo[BQ];
+    int hi[BQ];
+    float lse2[BQ];
+    float dv[BQ];
+};
+
+template <int D>
+struct Layout {
+    static constexpr int KB = D / 64;
+    static constexpr int K_OFF = 0;
+    static constexpr int V_OFF = K_OFF + KB * KTILE;
+    static constexpr int Q_OFF = V_OFF + KB * KTILE;             // 2 stages
+    static constexpr int DO_OFF = Q_OFF + 2 * KB * QTILE;        // 2 stages
+    static constexpr int BAND_OFF = DO_OFF + 2 * KB * QTILE;     // 2 buffers (one per warpgroup)
+    static constexpr int INFO_OFF = BAND_OFF + 2 * BAND_BYTES;   // 2 StepInfo
+    static constexpr int BAR_OFF = INFO_OFF + 2 * int(sizeof(StepInfo));
+    // kv_full, qd_full[2], qd_empty[2], s_full[2], p_full[2], acc_full, drain
+    static constexpr int NBARS = 11;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+    static constexpr int TOTAL = MISC_OFF + 64;
+    static constexpr int ALLOC = TOTAL + 1024;
+    static constexpr uint32_t DK_COL = 0;
+    static constexpr uint32_t DV_COL = D;
+    static constexpr uint32_t s_col(int bb) { return uint32_t(2 * D + 128 * bb); }
+    static constexpr uint32_t dp_col(int bb) { return uint32_t(2 * D + 128 * bb + 64); }
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const AttnParams p, const int num_ktiles) {
+    using L = Layout<D>;
+    constexpr int KB = L::KB;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* qd_full = bars + 1;   // [2]
+    uint64_t* qd_empty = bars + 3;  // [2]
+    uint64_t* s_full = bars + 5;    // [2]
+    uint64_t* p_full = bars + 7;    // [2]
+    uint64_t* acc_full = bars + 9;
+    uint64_t* drain = bars + 10;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
+    int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.Hq / p.Hkv;
+    const int kt = int(blockIdx.x) % num_ktiles;
+    const int bg = int(blockIdx.x) / num_ktiles;
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int j0 = kt * BK;
+    const int t64 = (p.S + 63) / 64;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&qd_full[u], 1);
+            mbar_init(&qd_empty[u], 1);
+            mbar_init(&s_full[u], 1);
+            mbar_init(&p_full[u], 4);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        ctl->abort = 0;
+        tinfo[0] = 0x7FFFFFFF;  // first query tile that sees the key tile
+        tinfo[1] = -1;          // last
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    // query tiles whose allowed key ranges intersect [j0, j0 + BK)
+    for (int t = threadIdx.x; t < t64; t += blockDim.x) {
+        const TileBounds tb = p.tile_bounds[size_t(b) * t64 + t];
+        if (tb.n_nonempty > 0 && tb.min_lo <= j0 + BK - 1 && tb.max_hi >= j0) {
+            atomicMin(&tinfo[0], t);
+            atomicMax(&tinfo[1], t);
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int qt_first = tinfo[0];
+    const int n_qt = (tinfo[1] >= tinfo[0]) ? tinfo[1] - tinfo[0] + 1 : 0;
+    const int n_steps = n_qt * G;
+
+    auto k_smem = [&](int kb) { return smem + L::K_OFF + kb * KTILE; };
+    auto v_smem = [&](int kb) { return smem + L::V_OFF + kb * KTILE; };
+    auto q_smem = [&](int st, int kb) { return smem + L::Q_OFF + (st * KB + kb) * QTILE; };
+    auto do_smem = [&](int st, int kb) { return smem + L::DO_OFF + (st * KB + kb) * QTILE; };
+    auto step_h = [&](int n) { return g * G + n / n_qt; };
+    auto step_qt = [&](int n) { return qt_first + n % n_qt; };
+
+    if (warp == TMA_WARP) {
+        if (lane == 0 && n_steps > 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_do);
+            mbar_arrive_expect_tx(kv_full, 2 * KB * KTILE);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_4d(k_smem(kb), &tm_k, kv_full, kb * 64, g, j0, b);
+                tma_load_4d(v_smem(kb), &tm_v, kv_full, kb * 64, g, j0, b);
+            }
+            int last = -1;
+            for (int n = 0; n < n_steps; ++n) {
+                const int st = n & 1;
+                if (!mbar_wait(&qd_empty[st], ((n >> 1) & 1) ^ 1, ctl, p.err, kErrDkdvQFree, p.timeout_ns)) break;
+                const int h = step_h(n), i0 = step_qt(n) * BQ;
+                mbar_arrive_expect_tx(&qd_full[st], 2 * KB * QTILE);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(q_smem(st, kb), &tm_q, &qd_full[st], kb * 64, h, i0, b);
+                    tma_load_4d(do_smem(st, kb), &tm_do, &qd_full[st], kb * 64, h, i0, b);
+                }
+                last = n;
+            }
+            mbar_wait_drain(kv_full, 0, p.timeout_ns);
+            for (int n = (last > 0 ? last - 1 : 0); n <= last; ++n)
+                if (n >= 0) mbar_wait_drain(&qd_full[n & 1], (n >> 1) & 1, p.timeout_ns);
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0 && n_steps > 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BQ, 0, 0);
+            constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
+            auto issue_sdp = [&](int n) {
+                const int st = n & 1, bb = n & 1;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int kb = kk >> 2, kin = kk & 3;
+                    const uint64_t ak = sdesc_sw128(smem_u32(k_smem(kb)) + kin * 32, 16, 1024);
+                    const uint64_t bq = sdesc_sw128(smem_u32(q_smem(st, kb)) + kin * 32, 16, 1024);
+                    mma_ss(tmem + L::s_col(bb), ak, bq, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int kb = kk >> 2, kin = kk & 3;
+                    const uint64_t av = sdesc_sw128(smem_u32(v_smem(kb)) + kin * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(smem_u32(do_smem(st, kb)) + kin * 32, 16, 1024);
+                    mma_ss(tmem + L::dp_col(bb), av, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[bb]);
+            };
+            bool ok = mbar_wait(kv_full, 0, ctl, p.err, kErrDkdvKV, p.timeout_ns) &&
+                      mbar_wait(&qd_full[0], 0, ctl, p.err, kErrDkdvQ, p.timeout_ns);
+            if (ok) {
+                tc_fence_after();
+                issue_sdp(0);
+            }
+            for (int n = 0; ok && n < n_steps; ++n) {
+                if (n + 1 < n_steps) {
+                    ok = mbar_wait(&qd_full[(n + 1) & 1], ((n + 1) >> 1) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_sdp(n + 1);
+                }
+                ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDkdvP, p.timeout_ns);
+                if (!ok) break;
+                tc_fence_after();
+                const int st = n & 1, bb = n & 1;
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk) {
+                    const uint64_t bdo = sdesc_sw128(smem_u32(do_smem(st, 0)) + kk * 2048, QTILE, 1024);
+                    mma_ts(tmem + L::DV_COL, tmem + L::s_col(bb) + kk * 8, bdo, IDESC_ACC,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk) {
+                    const uint64_t bq = sdesc_sw128(smem_u32(q_smem(st, 0)) + kk * 2048, QTILE, 1024);
+                    mma_ts(tmem + L::DK_COL, tmem + L::dp_col(bb) + kk * 8, bq, IDESC_ACC,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&qd_empty[st]);
+            }
+            if (ok) mma_commit(acc_full);
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------------ elementwise warpgroups
+        const int w = warp >> 2;       // this warpgroup takes steps n with n % 2 == w
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;  // key row (TMEM lane)
+        const int j = j0 + r;
+        const uint32_t lane_base = uint32_t(wq * 32) << 16;
+        const int tid = threadIdx.x & 127;
+        uint8_t* band = smem + L::BAND_OFF + w * BAND_BYTES;
+        StepInfo* info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF) + w;
+
+        // stage the profile band (query rows of the step, distance window) and row info
+        auto stage = [&](int n) {
+            const int h = step_h(n), i0 = step_qt(n) * BQ;
+            const int delta = p.q_off + i0 - j0;
+            for (int id = tid; id < BQ * BAND_CHUNKS; id += 128) {
+                const int c = id / BAND_CHUNKS, q = id % BAND_CHUNKS;
+                const int i = i0 + c;
+                const int m_c = (delta + c - 127) & 7;
+                const int d0 = delta + c - 127 - m_c + 8 * q;
+                const bool inb = p.R > 0 && i < p.S && d0 >= 0 && d0 < p.R;
+                const void* src = inb ? static_cast<const void*>(p.profiles +
+                                                                 ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) + d0)
+                                      : p.safe_src;
+                cp_async_16(smem_u32(band + c * BAND_PITCH + 16 * q), src, inb ? 16u : 0u);
+            }
+            cp_async_commit();
+            if (tid < BQ) {
+                const int i = i0 + tid;
+                int2 rb = make_int2(kEmptyLo, kEmptyHi);
+                float l2 = 0.f, dv = 0.f;
+                if (i < p.S) {
+                    rb = p.row_bounds[size_t(b) * p.S + i];
+                    const size_t t = (size_t(b) * p.Hq + h) * p.S + i;
+                    l2 = p.lse2t[t];
+                    dv = p.dvt[t];
+                }
+                info->lo[tid] = rb.x;
+                info->hi[tid] = rb.y;
+                info->lse2[tid] = l2;
+                info->dv[tid] = dv;
+            }
+        };
+
+        if (w < n_steps) stage(w);
+        bool ok = true;
+        for (int n = w; n < n_steps; n += 2) {
+            const int bb = n & 1;
+            const int h = step_h(n), qt = step_qt(n), i0 = qt * BQ;
+            const int delta = p.q_off + i0 - j0;
+            const TileBounds tb = p.tile_bounds[size_t(b) * t64 + qt];
+            const bool full = tb.n_nonempty == BQ && tb.max_lo <= j0 && tb.min_hi >= j0 + BK - 1;
+            // all four warps reach this vote whatever their wait returned, so the
+            // warpgroup leaves the loop together (the vote doubles as the barrier
+            // that publishes the staged band and row info)
+            const bool got = warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDkdvS, p.timeout_ns);
+            cp_async_wait_all();
+            if (!named_bar_and(1 + w, 128, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sv[64], dp[64];
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+            tmem_wait_ld();
+
+            float* dprow0 = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R);
+            uint32_t pk[32], dk[32];
+#pragma unroll
+            for (int c = 0; c < BQ; c += 2) {
+                float pv[2], ds[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int cc = c + u;
+                    const int d = delta + cc - r;
+                    const int m_c = (delta + cc - 127) & 7;
+                    const uint16_t braw =
+                        *reinterpret_cast<const uint16_t*>(band + cc * BAND_PITCH + 2 * (m_c + 127 - r));
+                    const float bias = __uint_as_float(uint32_t(braw) << 16);
+                    const bool allowed = full || (j >= info->lo[cc] && j <= info->hi[cc]);
+                    const float z2 = fmaf(__uint_as_float(sv[cc]), p.scale_log2, bias * kLog2e);
+                    const float pr = allowed ? ex2_approx(z2 - info->lse2[cc]) : 0.f;
+                    const float dsv = pr * (__uint_as_float(dp[cc]) - info->dv[cc]);
+                    if (allowed && d < p.R) dprow0[size_t(cc) * p.R + d] = dsv;
+                    pv[u] = pr;
+                    ds[u] = dsv;
+                }
+                pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+                dk[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+            }
+            tmem_st16(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            tmem_st16(tmem + lane_base + L::s_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[bb]);
+            named_bar_sync(1 + w, 128);  // band and info of this step fully consumed
+            if (n + 2 < n_steps) stage(n + 2);
+        }
+        cp_async_wait_all();
+
+        // ---- epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV ----
+        if (ok && n_steps > 0) {
+            ok = warp_wait(acc_full, 0, ctl, p.err, kErrDkdvAcc, p.timeout_ns);
+            tc_fence_after();
+        }
+        if (ok) {
+            const bool row_in = j < p.Skv;
+            float* dst = (w == 0 ? p.dk : p.dv) + ((size_t(b) * p.Skv + j) * p.Hkv + g) * size_t(D);
+            const float mul = (w == 0) ? p.scale : 1.f;
+            const uint32_t col = (w == 0) ? L::DK_COL : L::DV_COL;
+            if (n_steps > 0) {
+#pragma unroll 1
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + col + 32 * c4, o);
+                    tmem_wait_ld();
+                    if (row_in) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float4 v = make_float4(__uint_as_float(o[4 * q]) * mul, __uint_as_float(o[4 * q + 1]) * mul,
+                                                   __uint_as_float(o[4 * q + 2]) * mul,
+                                                   __uint_as_float(o[4 * q + 3]) * mul);
+                            *reinterpret_cast<float4*>(dst + 32 * c4 + 4 * q) = v;
+                        }
+                    }
+                }
+            } else if (row_in) {
+                for (int e = 0; e < D; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+template <int D>
+cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                   const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
+    using L = Layout<D>;
+    auto kern = dkdv_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    const int nkt = (p.Skv + BK - 1) / BK;
+    const long long grid = (long long)nkt * p.B * p.Hkv;
+    if (grid == 0) return cudaSuccess;
+    kern<<<dim3(unsigned(grid)), dim3(320), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nkt);
+    return cudaGetLastError();
+}
+
+}  // namespace kv
+
+// =====================================================================================
+// dQ
+// =====================================================================================
+namespace dqk {
+
+constexpr int BM = 128;               // query rows per CTA (TMEM lanes)
+constexpr int BN = 64;                // keys per step
+constexpr int BAND_CHUNKS = 9;        // 72 bf16 per row window
+constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
+constexpr int BAND_BYTES = BAND_UNITS * 16;
+constexpr int QTILE = BM * 128;       // [128 x 64 bf16]
+constexpr int KTILE = BN * 128;       // [64 x 64 bf16]
+
+__host__ __device__ constexpr int band_unit(int r) { return BAND_CHUNKS * r + 2 * (r >> 3); }
+
+template <int D>
+struct Layout {
+    static constexpr int KB = D / 64;
+    static constexpr int Q_OFF = 0;
+    static constexpr int DO_OFF = Q_OFF + KB * QTILE;
+    static constexpr int K_OFF = DO_OFF + KB * QTILE;        // 2 stages
+    static constexpr int V_OFF = K_OFF + 2 * KB * KTILE;     // 2 stages
+    static constexpr int BAND_OFF = V_OFF + 2 * KB * KTILE;  // 2 buffers (one per warpgroup)
+    static constexpr int BAR_OFF = BAND_OFF + 2 * BAND_BYTES;
+    // q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], acc_full, drain
+    static constexpr int NBARS = 11;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+    static constexpr int TOTAL = MISC_OFF + 64;
+    static constexpr int ALLOC = TOTAL + 1024;
+    static constexpr uint32_t DQ_COL = 0;
+    static constexpr uint32_t s_col(int bb) { return uint32_t(D + 128 * bb); }
+    static constexpr uint32_t dp_col(int bb) { return uint32_t(D + 128 * bb + 64); }
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const AttnParams p, const int num_qtiles) {
+    using L = Layout<D>;
+    constexpr int KB = L::KB;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* q_full = bars + 0;
+    uint64_t* kv_full = bars + 1;   // [2]
+    uint64_t* kv_empty = bars + 3;  // [2]
+    uint64_t* s_full = bars + 5;    // [2]
+    uint64_t* p_full = bars + 7;    // [2]
+    uint64_t* acc_full = bars + 9;
+    uint64_t* drain = bars + 10;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
+    int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per_tile = p.B * p.Hq;
+    const int qt = num_qtiles - 1 - int(blockIdx.x) / per_tile;
+    const int rem = int(blockIdx.x) % per_tile;
+    const int b = rem / p.Hq, h = rem % p.Hq;
+    const int g = h / (p.Hq / p.Hkv);
+    const int i0 = qt * BM;
+    const int i0g = p.q_off + i0;
+    const int t64 = (p.S + 63) / 64;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&kv_full[u], 1);
+            mbar_init(&kv_empty[u], 1);
+            mbar_init(&s_full[u], 1);
+            mbar_init(&p_full[u], 4);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        ctl->abort = 0;
+        const TileBounds* tb = p.tile_bounds + size_t(b) * t64 + 2 * qt;
+        int min_lo = tb[0].min_lo, max_hi = tb[0].max_hi, ne = tb[0].n_nonempty;
+        if (2 * qt + 1 < t64) {
+            min_lo = min(min_lo, tb[1].min_lo);
+            max_hi = max(max_hi, tb[1].max_hi);
+            ne += tb[1].n_nonempty;
+        }
+        int t_begin = 0, n_steps = 0;
+        if (ne > 0) {
+            // step t covers keys [i0g + 64 - 64 t, i0g + 127 - 64 t]
+            t_begin = max(0, ceil_div_i(i0g + BN - max_hi, BN));
+            const int t_end = floor_div(i0g + 2 * BN - 1 - min_lo, BN);
+            n_steps = max(0, t_end - t_begin + 1);
+        }
+        tinfo[0] = t_begin;
+        tinfo[1] = n_steps;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int t_begin = tinfo[0];
+    const int n_steps = tinfo[1];
+
+    auto q_smem = [&](int kb) { return smem + L::Q_OFF + kb * QTILE; };
+    auto do_smem = [&](int kb) { return smem + L::DO_OFF + kb * QTILE; };
+    auto k_smem = [&](int st, int kb) { return smem + L::K_OFF + (st * KB + kb) * KTILE; };
+    auto v_smem = [&](int st, int kb) { return smem + L::V_OFF + (st * KB + kb) * KTILE; };
+    auto key0 = [&](int n) { return i0g + BN - (t_begin + n) * BN; };
+
+    if (warp == TMA_WARP) {
+        if (lane == 0 && n_steps > 0) {
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_do);
+            mbar_arrive_expect_tx(q_full, 2 * KB * QTILE);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_4d(q_smem(kb), &tm_q, q_full, kb * 64, h, i0, b);
+                tma_load_4d(do_smem(kb), &tm_do, q_full, kb * 64, h, i0, b);
+            }
+            int last = -1;
+            for (int n = 0; n < n_steps; ++n) {
+                const int st = n & 1;
+                if (!mbar_wait(&kv_empty[st], ((n >> 1) & 1) ^ 1, ctl, p.err, kErrDqKVFree, p.timeout_ns)) break;
+                const int jk = key0(n);
+                mbar_arrive_expect_tx(&kv_full[st], 2 * KB * KTILE);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(k_smem(st, kb), &tm_k, &kv_full[st], kb * 64, g, jk, b);
+                    tma_load_4d(v_smem(st, kb), &tm_v, &kv_full[st], kb * 64, g, jk, b);
+                }
+                last = n;
+            }
+            mbar_wait_drain(q_full, 0, p.timeout_ns);
+            for (int n = (last > 0 ? last - 1 : 0); n <= last; ++n)
+                if (n >= 0) mbar_wait_drain(&kv_full[n & 1], (n >> 1) & 1, p.timeout_ns);
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0 && n_steps > 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
+            constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);
+            auto issue_sdp = [&](int n) {
+                const int st = n & 1, bb = n & 1;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int kb = kk >> 2, kin = kk & 3;
+                    const uint64_t aq = sdesc_sw128(smem_u32(q_smem(kb)) + kin * 32, 16, 1024);
+                    const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, kb)) + kin * 32, 16, 1024);
+                    mma_ss(tmem + L::s_col(bb), aq, bk, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int kb = kk >> 2, kin = kk & 3;
+                    const uint64_t ad = sdesc_sw128(smem_u32(do_smem(kb)) + kin * 32, 16, 1024);
+                    const uint64_t bv = sdesc_sw128(smem_u32(v_smem(st, kb)) + kin * 32, 16, 1024);
+                    mma_ss(tmem + L::dp_col(bb), ad, bv, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[bb]);
+            };
+            bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns) &&
+                      mbar_wait(&kv_full[0], 0, ctl, p.err, kErrDqKV, p.timeout_ns);
+            if (ok) {
+                tc_fence_after();
+                issue_sdp(0);
+            }
+            for (int n = 0; ok && n < n_steps; ++n) {
+                if (n + 1 < n_steps) {
+                    ok = mbar_wait(&kv_full[(n + 1) & 1], ((n + 1) >> 1) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_sdp(n + 1);
+                }
+                ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
+                if (!ok) break;
+                tc_fence_after();
+                const int st = n & 1, bb = n & 1;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, 0)) + kk * 2048, KTILE, 1024);
+                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + kk * 8, bk, IDESC_DQ,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&kv_empty[st]);
+            }
+            if (ok) mma_commit(acc_full);
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, p.timeout_ns);
+        }
+    } else {
+        const int w = warp >> 2;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_base = uint32_t(wq * 32) << 16;
+        const int i = i0 + r;
+        const bool row_in = i < p.S;
+        const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
+        const bool empty = rb.x > rb.y;
+        const size_t trow = (size_t(b) * p.Hq + h) * p.S + i;
+        const float lse2 = row_in ? p.lse2t[trow] : 0.f;
+        const float dvr = row_in ? p.dvt[trow] : 0.f;
+
+        uint8_t* band = smem + L::BAND_OFF + w * BAND_BYTES;
+        const int unit = band_unit(r);
+        const uint32_t band_saddr = smem_u32(band) + uint32_t(unit) * 16u;
+        const uint32_t* band_words = reinterpret_cast<const uint32_t*>(band + unit * 16);
+        const int m_r = (r + 1) & 7;
+        const int g_r = m_r >> 1;
+        const uint32_t fshift = uint32_t(m_r & 1) * 16u;
+        const uint16_t* prof_row =
+            (p.R > 0 && row_in && !empty) ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) : nullptr;
+        // step n has distance offset delta = i0g - key0(n) = 64 (t_begin + n) - 64
+        auto band_needed = [&](int n) { return BN * (t_begin + n) - BN + wq * 32 - (BN - 1) < p.R; };
+        auto issue_band = [&](int n) {
+            const int x0 = BN * (t_begin + n) - BN + r - (BN - 1) - m_r;
+#pragma unroll
+            for (int q = 0; q < BAND_CHUNKS; ++q) {
+                const int d0 = x0 + 8 * q;
+                const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
+                const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
+                cp_async_16(band_saddr + 16u * q, src, inb ? 16u : 0u);
+            }
+            cp_async_commit();
+        };
+
+        if (w < n_steps && band_needed(w)) issue_band(w);
+        bool ok = true;
+        for (int n = w; n < n_steps; n += 2) {
+            const int bb = n & 1;
+            const int jk = key0(n);
+            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + BN - 1);
+            const bool need_mask = !__all_sync(0xffffffffu, my_full);
+            const bool use_band = band_needed(n);
+            if (!warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDqS, p.timeout_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sv[64], dp[64];
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+            tmem_wait_ld();
+            uint32_t wv[33];
+            if (use_band) {
+                cp_async_wait_all();
+#pragma unroll
+                for (int q = 0; q < 33; ++q) wv[q] = band_words[g_r + q];
+            }
+            // the row's band buffer is free: prefetch the window of this warpgroup's next step
+            if (n + 2 < n_steps && band_needed(n + 2)) issue_band(n + 2);
+            uint32_t dk[32];
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) {
+                const int c = 2 * pp;
+                float b0 = 0.f, b1 = 0.f;
+                if (use_band) {
+                    const uint32_t v = funnel_r(wv[31 - pp], wv[32 - pp], fshift);
+                    b1 = bf16lo_to_f32(v);
+                    b0 = bf16hi_to_f32(v);
+                }
+                float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, fmaf(b0, kLog2e, -lse2)));
+                float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, fmaf(b1, kLog2e, -lse2)));
+                if (need_mask) {
+                    const int jj = jk + c;
+                    p0 = (jj >= rb.x && jj <= rb.y) ? p0 : 0.f;
+                    p1 = (jj + 1 >= rb.x && jj + 1 <= rb.y) ? p1 : 0.f;
+                }
+                const float d0v = p0 * (__uint_as_float(dp[c]) - dvr);
+                const float d1v = p1 * (__uint_as_float(dp[c + 1]) - dvr);
+                dk[pp] = pack_bf16x2(d0v, d1v);
+            }
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[bb]);
+        }
+        cp_async_wait_all();
+
+        // ---- epilogue: each warpgroup writes half of the dQ columns ----
+        if (ok && n_steps > 0) {
+            ok = warp_wait(acc_full, 0, ctl, p.err, kErrDqAcc, p.timeout_ns);
+            tc_fence_after();
+        }
+        if (ok) {
+            float* dst = p.dq + ((size_t(b) * p.S + i) * p.Hq + h) * size_t(D);
+            constexpr int HALF = D / 2;
+            if (n_steps > 0) {
+#pragma unroll 1
+                for (int c4 = 0; c4 < HALF / 32; ++c4) {
+                    const int col = w * HALF + 32 * c4;
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + L::DQ_COL + col, o);
+                    tmem_wait_ld();
+                    if (row_in) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float4 v;
+                            v.x = empty ? 0.f : __uint_as_float(o[4 * q]) * p.scale;
+                            v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * p.scale;
+                            v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * p.scale;
+                            v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * p.scale;
+                            *reinterpret_cast<float4*>(dst + col + 4 * q) = v;
+                        }
+                    }
+                }
+            } else if (row_in) {
+                for (int e = w * HALF; e < (w + 1) * HALF; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+template <int D>
+cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                   const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
+    using L = Layout<D>;
+    auto kern = dq_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    const int nqt = (p.S + BM - 1) / BM;
+    const long long grid = (long long)nqt * p.B * p.Hq;
+    if (grid == 0) return cudaSuccess;
+    kern<<<dim3(unsigned(grid)), dim3(320), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nqt);
+    return cudaGetLastError();
+}
+
+}  // namespace dqk
+}  // namespace bwdk
+
+cudaError_t launch_bwd_dkdv(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                            const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
+    return p.D == 128 ? bwdk::kv::launch<128>(tm_q, tm_k, tm_v, tm_do, p, st)
+                      : bwdk::kv::launch<64>(tm_q, tm_k, tm_v, tm_do, p, st);
+}
+
+cudaError_t launch_bwd_dq(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
+    return p.D == 128 ? bwdk::dqk::launch<128>(tm_q, tm_k, tm_v, tm_do, p, st)
+                      : bwdk::dqk::launch<64>(tm_q, tm_k, tm_v, tm_do, p, st);
+}
+
+}  // namespace ira

@@ -1,0 +1,389 @@
+// host.cu -- the C ABI of libinkling_rel_attn.so (declared in
+// include/inkling_rel_attn.h): argument checks, workspace carving, TMA
+// descriptor encoding and the launch sequence of each entry point.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "inkling_rel_attn.h"
+#include "launch.h"
+
+namespace {
+
+using namespace ira;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// BF16 tensor [B, T, H, D] as a 4-D map {D, H, T, B}; box {64, 1, rows, 1};
+// 128-byte swizzle; out-of-range rows read as zero.
+bool encode_bhtd(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t H, int64_t D, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+    cuuint64_t strides[3] = {cuuint64_t(D * 2), cuuint64_t(H * D * 2), cuuint64_t(T * H * D * 2)};
+    cuuint32_t box[4] = {64u, 1u, cuuint32_t(rows), 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Last CUDA error seen by an entry point of this thread (inkling_rel_attn_last_cuda_error).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+cudaError_t note(cudaError_t e) {
+    if (e != cudaSuccess) t_last_cuda_error = e;
+    return e;
+}
+
+// Optional per-launch timing events (inkling_rel_attn_set_timing_events).
+cudaEvent_t const* g_events = nullptr;
+int g_event_pairs = 0;
+
+struct LaunchTimer {
+    cudaStream_t st;
+    int k = 0;
+    explicit LaunchTimer(cudaStream_t s) : st(s) {}
+    cudaError_t record(int idx) {
+        return (g_events && k < g_event_pairs) ? note(cudaEventRecord(g_events[idx], st)) : cudaSuccess;
+    }
+    template <class F>
+    cudaError_t run(F&& f) {
+        cudaError_t e = record(2 * k);
+        if (e == cudaSuccess) e = note(f());
+        if (e == cudaSuccess) e = record(2 * k + 1);
+        ++k;
+        return e;
+    }
+};
+
+inkling_status check_dims(const inkling_rel_attn_dims* d) {
+    if (!d) return INKLING_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->seq_q < 0 || d->seq_k < 0 || d->heads_q <= 0 || d->heads_kv <= 0 ||
+        d->rel_extent < 0 || d->window < 0 || d->query_offset < 0)
+        return INKLING_ERR_INVALID_ARG;
+    if (d->heads_q % d->heads_kv != 0) return INKLING_ERR_INVALID_ARG;
+    if (d->head_dim != 64 && d->head_dim != 128) return INKLING_ERR_UNSUPPORTED;
+    if (d->rel_extent % 8 != 0) return INKLING_ERR_UNSUPPORTED;
+    const int64_t lim = int64_t(1) << 30;
+    if (d->seq_q >= lim || d->seq_k >= lim || d->query_offset >= lim || d->batch >= lim || d->heads_q >= 65536 ||
+        d->rel_extent >= lim || d->window >= lim)
+        return INKLING_ERR_UNSUPPORTED;
+    // grid sizes
+    const int64_t nqt = (d->seq_q + 127) / 128, nkt = (d->seq_k + 127) / 128;
+    if (nqt * d->batch * d->heads_q >= (int64_t(1) << 31) || nkt * d->batch * d->heads_kv >= (int64_t(1) << 31))
+        return INKLING_ERR_UNSUPPORTED;
+    return INKLING_OK;
+}
+
+struct Ws {
+    WorkspaceLayout L;
+    uint8_t* base;
+    int* ctl() const { return reinterpret_cast<int*>(base + L.ctl); }
+    int2* kspan() const { return reinterpret_cast<int2*>(base + L.kspan); }
+    int* edges() const { return reinterpret_cast<int*>(base + L.edges); }
+    int2* row_bounds() const { return reinterpret_cast<int2*>(base + L.row_bounds); }
+    TileBounds* tiles() const { return reinterpret_cast<TileBounds*>(base + L.tile_bounds); }
+};
+
+inkling_status get_ws(const inkling_rel_attn_dims* d, bool backward, void* ws, size_t bytes, Ws* out) {
+    out->L = workspace_layout(d->batch, d->seq_q, d->heads_q, d->head_dim, backward);
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < out->L.total) return INKLING_ERR_INVALID_ARG;
+    out->base = static_cast<uint8_t*>(ws);
+    return INKLING_OK;
+}
+
+// key_valid / key_positions defaults (Inkling2FlexAttention.forward: key_valid
+// defaults to valid, key positions to the query positions in the single-shard case).
+inkling_status resolve_key_side(const inkling_rel_attn_dims* d, const uint8_t* valid, const uint8_t*& key_valid,
+                                const int32_t* positions, const int32_t* key_positions, int* key_pos_from_query) {
+    const bool single = d->seq_k == d->seq_q && d->query_offset == 0;
+    if (!key_valid) {
+        if (!single) return INKLING_ERR_INVALID_ARG;
+        key_valid = valid;
+    }
+    *key_pos_from_query = 0;
+    if (!key_positions && positions) {
+        if (!single) return INKLING_ERR_INVALID_ARG;
+        *key_pos_from_query = 1;
+    }
+    return INKLING_OK;
+}
+
+inkling_status cuda_status(cudaError_t e) { return note(e) == cudaSuccess ? INKLING_OK : INKLING_ERR_CUDA; }
+
+AttnParams base_params(const inkling_rel_attn_dims* d, const Ws& w, const uint16_t* profiles, const float* sink) {
+    AttnParams p{};
+    p.B = int(d->batch);
+    p.S = int(d->seq_q);
+    p.Skv = int(d->seq_k);
+    p.Hq = int(d->heads_q);
+    p.Hkv = int(d->heads_kv);
+    p.D = int(d->head_dim);
+    p.R = int(d->rel_extent);
+    p.W = int(d->window);
+    p.q_off = int(d->query_offset);
+    p.scale = 1.0f / sqrtf(float(d->head_dim));
+    p.scale_log2 = p.scale * kLog2e;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.profiles = profiles;
+    p.safe_src = w.row_bounds();
+    p.sink = sink;
+    p.row_bounds = w.row_bounds();
+    p.tile_bounds = w.tiles();
+    p.err = w.ctl();
+    return p;
+}
+
+// Prologue shared by fwd and bwd: clear the error word, key span, row ranges.
+inkling_status run_bounds(const inkling_rel_attn_dims* d, const Ws& w, const uint8_t* valid,
+                          const uint8_t* key_valid, const int32_t* positions, cudaStream_t st, LaunchTimer& tm) {
+    cudaError_t e = cudaMemsetAsync(w.ctl(), 0, 16, st);
+    if (e == cudaSuccess)
+        e = tm.run([&] { return launch_kspan(key_valid, int(d->batch), int(d->seq_k), w.kspan(), st); });
+    if (e == cudaSuccess)
+        e = tm.run([&] {
+            return launch_bounds(valid, positions, w.kspan(), int(d->batch), int(d->seq_q), int(d->query_offset),
+                                 int(d->window), w.row_bounds(), w.tiles(), st);
+        });
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t inkling_rel_attn_workspace_size(const inkling_rel_attn_dims* dims, int backward) {
+    if (check_dims(dims) != INKLING_OK) return 0;
+    return workspace_layout(dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, backward != 0).total;
+}
+
+inkling_status inkling_rel_attn_validate(const inkling_rel_attn_dims* dims, const uint8_t* valid,
+                                         const uint8_t* key_valid, const int32_t* positions,
+                                         const int32_t* key_positions, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    if (!valid && dims->batch * dims->seq_q > 0) return INKLING_ERR_INVALID_ARG;
+    int kpq = 0;
+    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
+    if (s != INKLING_OK) return s;
+    if (!key_valid && dims->batch * dims->seq_k > 0) return INKLING_ERR_INVALID_ARG;
+    Ws w;
+    s = get_ws(dims, false, workspace, workspace_bytes, &w);
+    if (s != INKLING_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int B = int(dims->batch);
+    cudaError_t e = cudaMemsetAsync(w.ctl(), 0, 16, st);
+    if (e == cudaSuccess && B > 0) e = cudaMemsetAsync(w.edges(), 0, size_t(B) * 8, st);
+    if (e == cudaSuccess)
+        e = launch_validate(valid, key_valid, positions, key_positions, B, int(dims->seq_q), int(dims->seq_k),
+                            int(dims->query_offset), kpq, w.ctl(), w.edges(), st);
+    int ctl[4] = {0, 0, 0, 0};
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ctl, w.ctl(), 16, cudaMemcpyDeviceToHost, st);
+    int* edges = nullptr;
+    if (e == cudaSuccess && B > 0) {
+        edges = new int[size_t(B) * 2];
+        e = cudaMemcpyAsync(edges, w.edges(), size_t(B) * 8, cudaMemcpyDeviceToHost, st);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        delete[] edges;
+        return INKLING_ERR_CUDA;
+    }
+    bool bad = ctl[1] != 0;
+    for (int b = 0; b < B && !bad; ++b) bad = edges[2 * b] > 1 || edges[2 * b + 1] > 1;
+    delete[] edges;
+    return bad ? INKLING_ERR_MALFORMED_POSITIONS : INKLING_OK;
+}
+
+inkling_status inkling_rel_attn_fwd(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
+                                    const uint16_t* v, const uint16_t* profiles, const float* sink,
+                                    const uint8_t* valid, const uint8_t* key_valid, const int32_t* positions,
+                                    const int32_t* key_positions, float* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
+    if (nq > 0 && (!q || !sink || !valid || !out || !lse)) return INKLING_ERR_INVALID_ARG;
+    if (nq > 0 && dims->rel_extent > 0 && !profiles) return INKLING_ERR_INVALID_ARG;
+    if (nk > 0 && (!k || !v)) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out))
+        return INKLING_ERR_INVALID_ARG;
+    int kpq = 0;
+    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
+    if (s != INKLING_OK) return s;
+    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
+    Ws w;
+    s = get_ws(dims, false, workspace, workspace_bytes, &w);
+    if (s != INKLING_OK) return s;
+    if (nq == 0) return INKLING_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // K/V maps need at least one row; with no keys every row is empty and the
+    // kernel never reads them, so point them at q.
+    const bool no_keys = dims->seq_k == 0;
+    CUtensorMap tq, tk, tv;
+    if (!encode_bhtd(&tq, q, dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, 128) ||
+        !encode_bhtd(&tk, no_keys ? q : k, dims->batch, no_keys ? 1 : dims->seq_k,
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 128) ||
+        !encode_bhtd(&tv, no_keys ? q : v, dims->batch, no_keys ? 1 : dims->seq_k,
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 128))
+        return INKLING_ERR_CUDA;
+
+    LaunchTimer tm(st);
+    s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
+    if (s != INKLING_OK) return s;
+    AttnParams p = base_params(dims, w, profiles, sink);
+    p.out = out;
+    p.lse = lse;
+    return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+}
+
+inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
+                                    const uint16_t* v, const uint16_t* profiles, const float* sink,
+                                    const uint8_t* valid, const uint8_t* key_valid, const int32_t* positions,
+                                    const int32_t* key_positions, const float* out, const float* lse,
+                                    const float* dout, const float* dlse, float* dq, float* dk, float* dv,
+                                    float* dprofiles, float* dsink, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
+    if (nq > 0 && (!q || !sink || !valid || !out || !lse || !dout || !dq || !dsink)) return INKLING_ERR_INVALID_ARG;
+    if (nq > 0 && dims->rel_extent > 0 && (!profiles || !dprofiles)) return INKLING_ERR_INVALID_ARG;
+    if (nk > 0 && (!k || !v || !dk || !dv)) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dprofiles))
+        return INKLING_ERR_INVALID_ARG;
+    int kpq = 0;
+    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
+    if (s != INKLING_OK) return s;
+    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
+    Ws w;
+    s = get_ws(dims, true, workspace, workspace_bytes, &w);
+    if (s != INKLING_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (nq == 0) {
+        // no queries: every key gradient is zero
+        cudaError_t e = cudaSuccess;
+        if (nk > 0) {
+            const size_t bytes = size_t(nk) * dims->heads_kv * dims->head_dim * 4;
+            e = cudaMemsetAsync(dk, 0, bytes, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, st);
+        }
+        return cuda_status(e);
+    }
+    const bool no_keys = dims->seq_k == 0;
+    auto* dout_bf16 = reinterpret_cast<__nv_bfloat16*>(w.base + w.L.dout_bf16);
+    auto* lse2t = reinterpret_cast<float*>(w.base + w.L.lse2t);
+    auto* dvt = reinterpret_cast<float*>(w.base + w.L.dvt);
+    CUtensorMap tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64;
+    const int64_t B = dims->batch, S = dims->seq_q, Hq = dims->heads_q, D = dims->head_dim;
+    const int64_t Skv_m = no_keys ? 1 : dims->seq_k, Hkv_m = no_keys ? Hq : dims->heads_kv;
+    const void* kb = no_keys ? static_cast<const void*>(q) : k;
+    const void* vb = no_keys ? static_cast<const void*>(q) : v;
+    if (!encode_bhtd(&tq64, q, B, S, Hq, D, 64) || !encode_bhtd(&tq128, q, B, S, Hq, D, 128) ||
+        !encode_bhtd(&tdo64, dout_bf16, B, S, Hq, D, 64) || !encode_bhtd(&tdo128, dout_bf16, B, S, Hq, D, 128) ||
+        !encode_bhtd(&tk128, kb, B, Skv_m, Hkv_m, D, 128) || !encode_bhtd(&tv128, vb, B, Skv_m, Hkv_m, D, 128) ||
+        !encode_bhtd(&tk64, kb, B, Skv_m, Hkv_m, D, 64) || !encode_bhtd(&tv64, vb, B, Skv_m, Hkv_m, D, 64))
+        return INKLING_ERR_CUDA;
+
+    LaunchTimer tm(st);
+    s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
+    if (s != INKLING_OK) return s;
+    cudaError_t e = tm.run([&] {
+        return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
+                               lse2t, dvt, st);
+    });
+    if (e == cudaSuccess)
+        e = tm.run([&] {
+            return dims->rel_extent > 0 ? launch_dprof_zero(w.row_bounds(), int(B), int(S), int(Hq),
+                                                            int(dims->rel_extent), int(dims->query_offset),
+                                                            dprofiles, st)
+                                        : cudaSuccess;
+        });
+    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    AttnParams p = base_params(dims, w, profiles, sink);
+    p.lse2t = lse2t;
+    p.dvt = dvt;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dprofiles = dprofiles;
+    e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, p, st) : cudaSuccess; });
+    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    return cuda_status(tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st); }));
+}
+
+inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream) {
+    if (!workspace) return INKLING_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    if (word != 0) {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        return INKLING_ERR_TIMEOUT;
+    }
+    return INKLING_OK;
+}
+
+inkling_status inkling_rel_attn_selftest_wait_timeout(uint32_t timeout_us, void* workspace, size_t workspace_bytes,
+                                                      void* stream) {
+    if (!workspace || workspace_bytes < 16 || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+        return INKLING_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, 16, st);
+    if (e == cudaSuccess) e = launch_selftest_wait(uint64_t(timeout_us) * 1000ull, static_cast<int*>(workspace), st);
+    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    return inkling_rel_attn_last_device_error(workspace, stream);
+}
+
+inkling_status inkling_rel_attn_set_timing_events(void* const* events, int n_pairs) {
+    if (n_pairs < 0) return INKLING_ERR_INVALID_ARG;
+    g_events = reinterpret_cast<cudaEvent_t const*>(events);
+    g_event_pairs = events ? n_pairs : 0;
+    return INKLING_OK;
+}
+
+const char* inkling_rel_attn_last_cuda_error(void) {
+    return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
+
+const char* inkling_status_string(inkling_status status) {
+    switch (status) {
+        case INKLING_OK: return "ok";
+        case INKLING_ERR_INVALID_ARG: return "invalid argument";
+        case INKLING_ERR_UNSUPPORTED: return "unsupported configuration";
+        case INKLING_ERR_MALFORMED_POSITIONS: return "malformed validity masks or positions";
+        case INKLING_ERR_TIMEOUT: return "device-side wait timed out";
+        case INKLING_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

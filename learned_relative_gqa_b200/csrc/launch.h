@@ -1,0 +1,36 @@
+// launch.h -- host-side launchers of the CUDA path (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace ira {
+
+cudaError_t launch_kspan(const uint8_t* key_valid, int B, int Skv, int2* kspan, cudaStream_t st);
+cudaError_t launch_bounds(const uint8_t* valid, const int32_t* positions, const int2* kspan, int B, int S,
+                          int q_off, int W, int2* row_bounds, TileBounds* tiles, cudaStream_t st);
+cudaError_t launch_validate(const uint8_t* valid, const uint8_t* key_valid, const int32_t* positions,
+                            const int32_t* key_positions, int B, int S, int Skv, int q_off,
+                            int key_pos_from_query, int* ctl, int* edges, cudaStream_t st);
+cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const float* sink, const float* dout,
+                            const float* dlse, int B, int S, int Hq, float* dsink, __nv_bfloat16* dout_bf16,
+                            float* lse2t, float* dvt, cudaStream_t st);
+cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
+                              cudaStream_t st);
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st);
+
+// Forward attention. tm_q: {D, Hq, S, B} box {64,1,128,1}; tm_k / tm_v: {D, Hkv, Skv, B} box {64,1,128,1}.
+cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                       const AttnParams& p, cudaStream_t st);
+
+// Backward attention. dkdv: tm_k / tm_v box {64,1,128,1}, tm_q / tm_do box {64,1,64,1}.
+cudaError_t launch_bwd_dkdv(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                            const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st);
+// dq: tm_q / tm_do box {64,1,128,1}, tm_k / tm_v box {64,1,64,1}.
+cudaError_t launch_bwd_dq(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st);
+
+}  // namespace ira

@@ -1,0 +1,339 @@
+// prep_kernels.cu -- the O(B*S) kernels around the attention kernels:
+//   * key span (first / last valid key column of each batch row),
+//   * per-row allowed key range [lo, hi] and per-64-row tile summaries,
+//   * the precondition checker behind inkling_rel_attn_validate,
+//   * the backward preprocessing (row dot products, dsink, BF16 copy of dout,
+//     log2-scaled lse),
+//   * zeroing of the dprofiles entries that no allowed key reaches.
+//
+// Row range. Under the preconditions (one contiguous valid span per row,
+// positions consecutive inside a document and restarting at 0), the keys a
+// valid query row i (global column i_g) may attend form one interval:
+//   lo = max(i_g - positions[i], first valid key, i_g - W + 1 if W > 0)
+//   hi = min(i_g, last valid key)
+// i_g - positions[i] is the column where the row's document starts
+// ("positions ... reset per document" on the Inkling2FlexAttention.forward
+// page), so the interval is exactly the causal, same-document, in-window,
+// valid keys of the definition.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace ira {
+
+namespace {
+
+__device__ __forceinline__ int warp_min(int v) {
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ int warp_max(int v) {
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ int warp_sum(int v) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace
+
+// grid (B), block 256
+__global__ void kspan_kernel(const uint8_t* __restrict__ key_valid, int Skv, int2* __restrict__ kspan) {
+    const int b = blockIdx.x;
+    int first = 0x7FFFFFFF, last = -1;
+    for (int j = threadIdx.x; j < Skv; j += blockDim.x) {
+        if (key_valid[size_t(b) * Skv + j]) {
+            first = min(first, j);
+            last = max(last, j);
+        }
+    }
+    __shared__ int sf[32], sl[32];
+    first = warp_min(first);
+    last = warp_max(last);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) { sf[w] = first; sl[w] = last; }
+    __syncthreads();
+    if (w == 0) {
+        const int nw = blockDim.x >> 5;
+        first = lane < nw ? sf[lane] : 0x7FFFFFFF;
+        last = lane < nw ? sl[lane] : -1;
+        first = warp_min(first);
+        last = warp_max(last);
+        if (lane == 0) kspan[b] = make_int2(first, last);
+    }
+}
+
+// grid (ceil(S/64), B), block 64
+__global__ void bounds_kernel(const uint8_t* __restrict__ valid, const int32_t* __restrict__ positions,
+                              const int2* __restrict__ kspan, int S, int q_off, int W,
+                              int2* __restrict__ row_bounds, TileBounds* __restrict__ tiles) {
+    const int b = blockIdx.y, tile = blockIdx.x, r = threadIdx.x;
+    const int i = tile * 64 + r;
+    const int2 ks = kspan[b];
+    int lo = kEmptyLo, hi = kEmptyHi;
+    const bool in_range = i < S;
+    if (in_range && valid[size_t(b) * S + i] && ks.x <= ks.y) {
+        const int ig = q_off + i;
+        const int pos = positions ? positions[size_t(b) * S + i] : ig;
+        int l = max(ig - pos, ks.x);
+        if (W > 0) l = max(l, ig - W + 1);
+        const int h = min(ig, ks.y);
+        if (l <= h) { lo = l; hi = h; }
+    }
+    if (in_range) row_bounds[size_t(b) * S + i] = make_int2(lo, hi);
+    const bool ne = lo <= hi;
+    int a_min_lo = ne ? lo : 0x7FFFFFFF, a_max_hi = ne ? hi : -0x7FFFFFFF;
+    int a_max_lo = ne ? lo : -0x7FFFFFFF, a_min_hi = ne ? hi : 0x7FFFFFFF;
+    int cnt = ne ? 1 : 0;
+    a_min_lo = warp_min(a_min_lo);
+    a_max_hi = warp_max(a_max_hi);
+    a_max_lo = warp_max(a_max_lo);
+    a_min_hi = warp_min(a_min_hi);
+    cnt = warp_sum(cnt);
+    __shared__ int red[2][5];
+    const int w = r >> 5;
+    if ((r & 31) == 0) {
+        red[w][0] = a_min_lo; red[w][1] = a_max_hi; red[w][2] = a_max_lo; red[w][3] = a_min_hi; red[w][4] = cnt;
+    }
+    __syncthreads();
+    if (r == 0) {
+        TileBounds t;
+        t.min_lo = min(red[0][0], red[1][0]);
+        t.max_hi = max(red[0][1], red[1][1]);
+        t.max_lo = max(red[0][2], red[1][2]);
+        t.min_hi = min(red[0][3], red[1][3]);
+        t.n_nonempty = red[0][4] + red[1][4];
+        t.n_rows = min(64, S - tile * 64);
+        t.pad0 = t.pad1 = 0;
+        tiles[size_t(b) * gridDim.x + tile] = t;
+    }
+}
+
+// Precondition checker. grid-stride over (b, column) of the longer of the two
+// streams; counts violations in ctl[1] and rising edges of the valid masks.
+__global__ void validate_kernel(const uint8_t* __restrict__ valid, const uint8_t* __restrict__ key_valid,
+                                const int32_t* __restrict__ positions, const int32_t* __restrict__ key_positions,
+                                int B, int S, int Skv, int q_off, int key_pos_from_query,
+                                int* __restrict__ ctl, int* __restrict__ edges) {
+    const int64_t T = S > Skv ? S : Skv;
+    const int64_t n = int64_t(B) * T;
+    int bad = 0;
+    for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < n; t += int64_t(gridDim.x) * blockDim.x) {
+        const int b = int(t / T), c = int(t % T);
+        // query side
+        if (c < S) {
+            const size_t o = size_t(b) * S + c;
+            const bool v = valid[o] != 0;
+            const bool vp = c > 0 && valid[o - 1] != 0;
+            if (v && !vp) atomicAdd(&edges[2 * b + 0], 1);
+            const int p = positions ? positions[o] : q_off + c;
+            if (v) {
+                if (p < 0) ++bad;
+                if (vp) {
+                    const int pp = positions ? positions[o - 1] : q_off + c - 1;
+                    if (!(p == pp + 1 || p == 0)) ++bad;
+                }
+            }
+            const int j = q_off + c;
+            if (j < Skv) {
+                const size_t ok = size_t(b) * Skv + j;
+                const bool kv = key_valid[ok] != 0;
+                if (kv != v) ++bad;
+                if (v) {
+                    const int kp = key_positions ? key_positions[ok] : (key_pos_from_query ? p : j);
+                    if (kp != p) ++bad;
+                }
+            } else if (v) {
+                ++bad;  // a valid query outside the key stream
+            }
+        }
+        // key side
+        if (c < Skv) {
+            const size_t o = size_t(b) * Skv + c;
+            const bool v = key_valid[o] != 0;
+            const bool vp = c > 0 && key_valid[o - 1] != 0;
+            if (v && !vp) atomicAdd(&edges[2 * b + 1], 1);
+            if (v) {
+                auto kpos = [&](int col) {
+                    if (key_positions) return key_positions[size_t(b) * Skv + col];
+                    if (key_pos_from_query) return positions ? positions[size_t(b) * S + col] : q_off + col;
+                    return col;
+                };
+                const int p = kpos(c);
+                if (p < 0) ++bad;
+                if (vp) {
+                    const int pp = kpos(c - 1);
+                    if (!(p == pp + 1 || p == 0)) ++bad;
+                }
+            }
+        }
+    }
+    if (bad) atomicAdd(&ctl[1], bad);
+}
+
+// Backward preprocessing: one warp per (b, i, h) row.
+template <int D>
+__global__ void bwd_prep_kernel(const float* __restrict__ out, const float* __restrict__ lse,
+                                const float* __restrict__ sink, const float* __restrict__ dout,
+                                const float* __restrict__ dlse, int B, int S, int Hq,
+                                float* __restrict__ dsink, __nv_bfloat16* __restrict__ dout_bf16,
+                                float* __restrict__ lse2t, float* __restrict__ dvt) {
+    constexpr int PER = D / 32;
+    const int64_t nrows = int64_t(B) * S * Hq;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t row = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows; row += warps) {
+        const float* o = out + row * D + lane * PER;
+        const float* g = dout + row * D + lane * PER;
+        float acc = 0.f;
+        float gv[PER];
+        if constexpr (PER == 4) {
+            const float4 a = *reinterpret_cast<const float4*>(o);
+            const float4 c = *reinterpret_cast<const float4*>(g);
+            gv[0] = c.x; gv[1] = c.y; gv[2] = c.z; gv[3] = c.w;
+            acc = a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+        } else {
+            const float2 a = *reinterpret_cast<const float2*>(o);
+            const float2 c = *reinterpret_cast<const float2*>(g);
+            gv[0] = c.x; gv[1] = c.y;
+            acc = a.x * c.x + a.y * c.y;
+        }
+        for (int of = 16; of > 0; of >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, of);
+        __nv_bfloat16* gb = dout_bf16 + row * D + lane * PER;
+        if constexpr (PER == 4) {
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(gv[0], gv[1]);
+            __nv_bfloat162 p1 = __floats2bfloat162_rn(gv[2], gv[3]);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&p0);
+            u.y = *reinterpret_cast<uint32_t*>(&p1);
+            *reinterpret_cast<uint2*>(gb) = u;
+        } else {
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(gv[0], gv[1]);
+            *reinterpret_cast<__nv_bfloat162*>(gb) = p0;
+        }
+        if (lane == 0) {
+            const float dv = acc - (dlse ? dlse[row] : 0.f);
+            const float l = lse[row], s = sink[row];
+            float ps = 0.f;
+            if (isfinite(l)) ps = expf(s - l);
+            else if (l == INFINITY && s == INFINITY) ps = 1.f;
+            dsink[row] = -ps * dv;
+            const int h = int(row % Hq);
+            const int64_t bi = row / Hq;
+            const int i = int(bi % S), b = int(bi / S);
+            const size_t t = (size_t(b) * Hq + h) * S + i;
+            lse2t[t] = l * kLog2e;
+            dvt[t] = dv;
+        }
+    }
+}
+
+// Zero the dprofiles entries of each (b, h, i) row that no allowed key
+// reaches: everything outside the visited distances [i_g - hi, i_g - lo].
+// One warp per row.
+__global__ void dprof_zero_kernel(const int2* __restrict__ row_bounds, int B, int S, int Hq, int R, int q_off,
+                                  float* __restrict__ dprof) {
+    const int64_t nrows = int64_t(B) * Hq * S;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t row = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows; row += warps) {
+        const int i = int(row % S);
+        const int b = int(row / (int64_t(S) * Hq));
+        const int2 bh = row_bounds[size_t(b) * S + i];
+        const int ig = q_off + i;
+        int dlo = R, dhi = -1;  // visited distances (inclusive); empty by default
+        if (bh.x <= bh.y) {
+            dlo = max(0, ig - bh.y);
+            dhi = min(R - 1, ig - bh.x);
+        }
+        float* base = dprof + row * int64_t(R);
+        for (int e0 = lane * 4; e0 < R; e0 += 128) {
+            const bool all_out = (e0 + 3 < dlo) || (e0 > dhi);
+            if (all_out) {
+                *reinterpret_cast<float4*>(base + e0) = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u;
+                    if (e < dlo || e > dhi) base[e] = 0.f;
+                }
+            }
+        }
+    }
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing
+// arrives on; the guard must give up after timeout_ns and record the site.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, int* err) {
+    __shared__ uint64_t bar;
+    __shared__ CtaControl ctl;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        ctl.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &ctl, err, kErrSelftest, timeout_ns);
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_kspan(const uint8_t* key_valid, int B, int Skv, int2* kspan, cudaStream_t st) {
+    if (B == 0) return cudaSuccess;
+    kspan_kernel<<<B, 256, 0, st>>>(key_valid, Skv, kspan);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bounds(const uint8_t* valid, const int32_t* positions, const int2* kspan, int B, int S,
+                          int q_off, int W, int2* row_bounds, TileBounds* tiles, cudaStream_t st) {
+    if (B == 0 || S == 0) return cudaSuccess;
+    dim3 grid((S + 63) / 64, B);
+    bounds_kernel<<<grid, 64, 0, st>>>(valid, positions, kspan, S, q_off, W, row_bounds, tiles);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_validate(const uint8_t* valid, const uint8_t* key_valid, const int32_t* positions,
+                            const int32_t* key_positions, int B, int S, int Skv, int q_off,
+                            int key_pos_from_query, int* ctl, int* edges, cudaStream_t st) {
+    const long long n = (long long)B * (S > Skv ? S : Skv);
+    if (n == 0) return cudaSuccess;
+    const int blocks = int(n / 256 + 1 < 4096 ? n / 256 + 1 : 4096);
+    validate_kernel<<<blocks, 256, 0, st>>>(valid, key_valid, positions, key_positions, B, S, Skv, q_off,
+                                            key_pos_from_query, ctl, edges);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const float* sink, const float* dout,
+                            const float* dlse, int B, int S, int Hq, float* dsink, __nv_bfloat16* dout_bf16,
+                            float* lse2t, float* dvt, cudaStream_t st) {
+    const long long rows = (long long)B * S * Hq;
+    if (rows == 0) return cudaSuccess;
+    const int blocks = int(rows / 8 + 1 < 148 * 32 ? rows / 8 + 1 : 148 * 32);
+    if (D == 128)
+        bwd_prep_kernel<128><<<blocks, 256, 0, st>>>(out, lse, sink, dout, dlse, B, S, Hq, dsink, dout_bf16, lse2t, dvt);
+    else
+        bwd_prep_kernel<64><<<blocks, 256, 0, st>>>(out, lse, sink, dout, dlse, B, S, Hq, dsink, dout_bf16, lse2t, dvt);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
+                              cudaStream_t st) {
+    const long long rows = (long long)B * S * Hq;
+    if (rows == 0 || R == 0) return cudaSuccess;
+    const int blocks = int(rows / 8 + 1 < 148 * 32 ? rows / 8 + 1 : 148 * 32);
+    dprof_zero_kernel<<<blocks, 256, 0, st>>>(row_bounds, B, S, Hq, R, q_off, dprof);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st) {
+    selftest_wait_kernel<<<1, 32, 0, st>>>(timeout_ns, err);
+    return cudaGetLastError();
+}
+
+}  // namespace ira

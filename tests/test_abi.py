@@ -1,0 +1,115 @@
+"""CPU-only checks of the C-ABI library: it builds, loads, exports every entry
+point declared in include/inkling_rel_attn.h, sizes workspaces, and rejects bad
+arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "inkling_rel_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from learned_relative_gqa_b200 import build, binding
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(inkling_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("inkling_rel_attn_fwd", "inkling_rel_attn_bwd", "inkling_rel_attn_validate",
+                 "inkling_rel_attn_workspace_size", "inkling_rel_attn_last_device_error", "inkling_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_library_does_not_link_the_oracle(lib):
+    from learned_relative_gqa_b200 import binding
+    data = open(binding.LIB_PATH, "rb").read()
+    assert b"oracle_fwd_f64" not in data and b"oracle_bwd_f64" not in data
+
+
+def dims(**kw):
+    from learned_relative_gqa_b200.binding import Dims
+    base = dict(batch=2, seq_q=256, seq_k=256, heads_q=8, heads_kv=2, head_dim=128, rel_extent=64, window=0,
+                query_offset=0)
+    base.update(kw)
+    return Dims(**base)
+
+
+def test_workspace_size(lib):
+    from learned_relative_gqa_b200.binding import inkling_rel_attn_workspace_size as ws
+    f, b = ws(dims(), False), ws(dims(), True)
+    assert 0 < f < b
+    # backward holds a BF16 copy of dout plus two [B,Hq,S] fp32 arrays
+    assert b - f >= 2 * 256 * 8 * 128 * 2 + 2 * 2 * 8 * 256 * 4
+    assert ws(dims(seq_q=512, seq_k=512), False) > f
+    assert ws(dims(head_dim=96), False) == 0
+    assert ws(dims(heads_q=6, heads_kv=4), False) == 0
+    assert ws(dims(rel_extent=12), False) == 0
+
+
+@pytest.mark.parametrize("bad,expect", [
+    (dict(head_dim=96), 2),
+    (dict(rel_extent=12), 2),
+    (dict(heads_q=6, heads_kv=4), 1),
+    (dict(window=-1), 1),
+    (dict(seq_q=-3), 1),
+])
+def test_fwd_rejects_bad_dims_on_host(lib, bad, expect):
+    d = dims(**bad)
+    st = lib.inkling_rel_attn_fwd(ctypes.byref(d), *([None] * 11), None, 0, None)
+    assert st == expect
+
+
+def test_fwd_rejects_null_and_misaligned_pointers(lib):
+    d = dims()
+    fake = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+    args = [fake] * 11
+    st = lib.inkling_rel_attn_fwd(ctypes.byref(d), None, *args[1:], fake, 1 << 30, None)
+    assert st == 1  # null q
+    st = lib.inkling_rel_attn_fwd(ctypes.byref(d), mis, *args[1:], fake, 1 << 30, None)
+    assert st == 1  # misaligned q
+    # workspace too small
+    st = lib.inkling_rel_attn_fwd(ctypes.byref(d), *args, fake, 16, None)
+    assert st == 1
+    # key_valid may not default to valid under a query offset
+    d2 = dims(query_offset=64, seq_k=320)
+    a2 = list(args)
+    a2[6] = None  # key_valid
+    st = lib.inkling_rel_attn_fwd(ctypes.byref(d2), *a2, fake, 1 << 30, None)
+    assert st == 1
+
+
+def test_bwd_rejects_bad_arguments_on_host(lib):
+    d = dims(head_dim=32)
+    assert lib.inkling_rel_attn_bwd(ctypes.byref(d), *([None] * 18), None, 0, None) == 2
+    d = dims()
+    fake = ctypes.c_void_p(0x10000)
+    args = [fake] * 18
+    args[13] = None  # dlse is optional
+    a = list(args)
+    a[14] = None     # dq missing
+    assert lib.inkling_rel_attn_bwd(ctypes.byref(d), *a, fake, 1 << 34, None) == 1
+
+
+def test_status_strings(lib):
+    from learned_relative_gqa_b200 import binding
+    assert binding.status_string(0) == "ok"
+    assert "timed out" in binding.status_string(4)
+    assert binding.status_string(77) == "unknown status"
