@@ -140,6 +140,37 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims,
                                     float* dq, float* dk, float* dv, float* dprofiles, float* dsink,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code that only receives its input and output
+ * buffers from a host framework (a plugin or custom-operator interface with no
+ * allocator to call), or code that must not call cudaMalloc because it can
+ * synchronise the device and stall unrelated work. Same arguments and results
+ * as inkling_rel_attn_fwd, minus the workspace; this call allocates nothing
+ * (no cudaMalloc / cudaFree, no allocating library routine).
+ * Not a counterpart of anything on the Inkling2 pages: an addition of this
+ * library.
+ *   - Scratch lives in one 4 MiB array of device memory inside the library,
+ *     present on every GPU that loads it until the process exits. The forward
+ *     needs about 8.5 bytes per (batch, query) token, so B * S up to roughly
+ *     480,000 fits; larger problems return INKLING_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the array and it keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other host
+ *     threads) race on it, so serialise them.
+ *   - A device-side wait that runs out is recorded inside that array, which
+ *     callers cannot hand to inkling_rel_attn_last_device_error; the outputs of
+ *     such a call are unspecified.
+ */
+inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims,
+                                            const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const uint16_t* profiles, const float* sink,
+                                            const uint8_t* valid, const uint8_t* key_valid,
+                                            const int32_t* positions, const int32_t* key_positions,
+                                            float* out, float* lse, void* stream);
+
 /* SYNCHRONOUS: waits on stream, returns INKLING_ERR_TIMEOUT if a kernel of the
  * last fwd/bwd call on this workspace gave up a bounded wait (and clears the
  * record), INKLING_OK otherwise. */

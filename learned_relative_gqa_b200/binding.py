@@ -60,6 +60,8 @@ def load(path: str = LIB_PATH):
     lib.inkling_rel_attn_fwd.argtypes = [dp] + [vp] * 11 + [vp, sz, vp]
     lib.inkling_rel_attn_bwd.restype = ctypes.c_int
     lib.inkling_rel_attn_bwd.argtypes = [dp] + [vp] * 18 + [vp, sz, vp]
+    lib.inkling_rel_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.inkling_rel_attn_fwd_noalloc.argtypes = [dp] + [vp] * 11 + [vp]
     lib.inkling_rel_attn_last_device_error.restype = ctypes.c_int
     lib.inkling_rel_attn_last_device_error.argtypes = [vp, vp]
     lib.inkling_rel_attn_selftest_wait_timeout.restype = ctypes.c_int
@@ -139,6 +141,18 @@ def inkling_rel_attn_bwd(dims: Dims, q, k, v, profiles, sink, valid, key_valid, 
         _p(positions), _p(key_positions), _p(out), _p(lse), _p(dout), _p(dlse), _p(dq), _p(dk), _p(dv),
         _p(dprofiles), _p(dsink), _p(workspace), workspace.numel(), _stream(stream))
     _check(st, "inkling_rel_attn_bwd")
+
+
+def inkling_rel_attn_fwd_noalloc(dims: Dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions,
+                                 out, lse, stream=None) -> int:
+    """Forward that uses the library's own static device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory. Returns the library status
+    (INKLING_ERR_UNSUPPORTED when the problem needs more than the 4 MiB of scratch).
+    """
+    return int(load().inkling_rel_attn_fwd_noalloc(
+        ctypes.byref(dims), _p(q), _p(k), _p(v), _p(profiles), _p(sink), _p(_u8(valid)), _p(_u8(key_valid)),
+        _p(positions), _p(key_positions), _p(out), _p(lse), _stream(stream)))
 
 
 def inkling_rel_attn_last_device_error(workspace, stream=None) -> int:

@@ -12,6 +12,13 @@
 #include "inkling_rel_attn.h"
 #include "launch.h"
 
+// Scratch of inkling_rel_attn_fwd_noalloc: a fixed-size array in device
+// memory that exists on every GPU that loads this library, for as long as the
+// process lives. Host code must not take its address directly (the name is a
+// host-side stand-in); it asks the runtime for the device address instead.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 using namespace ira;
@@ -168,6 +175,28 @@ inkling_status run_bounds(const inkling_rel_attn_dims* d, const Ws& w, const uin
                                  int(d->window), w.row_bounds(), w.tiles(), st);
         });
     return cuda_status(e);
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (with that device current) and cached.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+inkling_status noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = note(cudaGetDevice(&dev));
+    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return INKLING_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = note(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+        if (e != cudaSuccess || !p) return INKLING_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return INKLING_OK;
 }
 
 }  // namespace
@@ -335,6 +364,25 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, p, st) : cudaSuccess; });
     if (e != cudaSuccess) return INKLING_ERR_CUDA;
     return cuda_status(tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st); }));
+}
+
+inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
+                                            const uint16_t* v, const uint16_t* profiles, const float* sink,
+                                            const uint8_t* valid, const uint8_t* key_valid,
+                                            const int32_t* positions, const int32_t* key_positions, float* out,
+                                            float* lse, void* stream) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    if (workspace_layout(dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, false).total >
+        kNoAllocScratchBytes)
+        return INKLING_ERR_UNSUPPORTED;  // problem needs more scratch than the static array holds
+    void* scratch = nullptr;
+    s = noalloc_scratch(&scratch);
+    if (s != INKLING_OK) return s;
+    // the ordinary forward, with the static array as its workspace (it clears the
+    // device error word itself and rewrites every other scratch byte it reads)
+    return inkling_rel_attn_fwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse,
+                                scratch, kNoAllocScratchBytes, stream);
 }
 
 inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream) {
