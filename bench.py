@@ -357,6 +357,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="train")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override the workload's sequence length (smaller cases for profiling)")
     ap.add_argument("--long-steps", type=int, default=3, help="forward steps of the long workload (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -367,7 +369,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from learned_relative_gqa_b200 import workloads
+    import dataclasses
     w = workloads.BY_NAME[args.workload]
+    if args.seq > 0:
+        w = dataclasses.replace(w, seq=args.seq)
     backward = w.backward
     if args.impl == "reference":
         # the oracle on the host cores; under torchrun only rank 0 works
@@ -392,7 +397,7 @@ def main():
     from learned_relative_gqa_b200 import binding, build
     build.build()
     binding.load()
-    x = workloads.make_inputs(w, device, seed=workloads.seed_of(w) + 7919 * rank)
+    x = workloads.make_inputs(w, device, seed=workloads.seed_of(workloads.BY_NAME[args.workload]) + 7919 * rank)
     D = w.head_dim
     E = workloads.allowed_counts(w, x)
     Ep = count_ep(x, E)

@@ -76,7 +76,7 @@ struct Layout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const AttnParams p, const int num_ktiles) {
@@ -148,6 +148,11 @@ __global__ void __launch_bounds__(320, 1)
     auto step_h = [&](int n) { return g * G + n / n_qt; };
     auto step_qt = [&](int n) { return qt_first + n % n_qt; };
 
+    // Launched with 384 x 168 registers; warpgroup 2 (producer, MMA issuer, two idle
+    // warps) gives its share to the two elementwise warpgroups
+    // (128 x 40 + 256 x 232 = 384 x 168). Each change sits at the top of its branch.
+    if (warp >= 8) {
+        setmaxnreg_dec<40>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -232,7 +237,9 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
         }
+    }
     } else {
+        setmaxnreg_inc<232>();
         // ------------------------------------------------------------ elementwise warpgroups
         const int w = warp >> 2;       // this warpgroup takes steps n with n % 2 == w
         const int wq = warp & 3;
@@ -301,29 +308,57 @@ __global__ void __launch_bounds__(320, 1)
             tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
             tmem_wait_ld();
 
-            float* dprow0 = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R);
+            // Band reads. Column cc reads element (m_cc + 127 - r) of band row cc, where
+            // m_cc = (delta + cc - 127) mod 8 repeats every 8 columns: eight per-step
+            // base pointers (one per cc mod 8) plus compile-time offsets cover them all.
+            const int dm = (delta - 127) & 7;
+            const uint16_t* bptr[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                bptr[u] = reinterpret_cast<const uint16_t*>(band + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r));
+            // dprofiles[b, h, i0 + c, delta + c - r] lives at dst0 + c * (R + 1)
+            float* dst0 = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) + (delta - r);
+            const size_t dstride = size_t(p.R) + 1;
+            const bool all_in_extent = delta + BQ - 1 < p.R;  // every distance of the step is < R
+            const int extent_left = p.R - delta;               // d < R  <=>  c - r < extent_left
+            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 l2e = make_float2(kLog2e, kLog2e);
             uint32_t pk[32], dk[32];
 #pragma unroll
-            for (int c = 0; c < BQ; c += 2) {
-                float pv[2], ds[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int cc = c + u;
-                    const int d = delta + cc - r;
-                    const int m_c = (delta + cc - 127) & 7;
-                    const uint16_t braw =
-                        *reinterpret_cast<const uint16_t*>(band + cc * BAND_PITCH + 2 * (m_c + 127 - r));
-                    const float bias = __uint_as_float(uint32_t(braw) << 16);
-                    const bool allowed = full || (j >= info->lo[cc] && j <= info->hi[cc]);
-                    const float z2 = fmaf(__uint_as_float(sv[cc]), p.scale_log2, bias * kLog2e);
-                    const float pr = allowed ? ex2_approx(z2 - info->lse2[cc]) : 0.f;
-                    const float dsv = pr * (__uint_as_float(dp[cc]) - info->dv[cc]);
-                    if (allowed && d < p.R) dprow0[size_t(cc) * p.R + d] = dsv;
-                    pv[u] = pr;
-                    ds[u] = dsv;
+            for (int c4 = 0; c4 < BQ / 4; ++c4) {
+                const float4 L4 = reinterpret_cast<const float4*>(info->lse2)[c4];  // broadcast reads
+                const float4 V4 = reinterpret_cast<const float4*>(info->dv)[c4];
+                int4 lo4 = make_int4(0, 0, 0, 0), hi4 = make_int4(0, 0, 0, 0);
+                if (!full) {
+                    lo4 = reinterpret_cast<const int4*>(info->lo)[c4];
+                    hi4 = reinterpret_cast<const int4*>(info->hi)[c4];
                 }
-                pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-                dk[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int c = 4 * c4 + 2 * h2;
+                    const float b0 = __uint_as_float(uint32_t(bptr[c & 7][1088 * (c >> 3)]) << 16);
+                    const float b1 = __uint_as_float(uint32_t(bptr[(c + 1) & 7][1088 * ((c + 1) >> 3)]) << 16);
+                    const float2 nl = h2 ? make_float2(-L4.z, -L4.w) : make_float2(-L4.x, -L4.y);
+                    const float2 nv = h2 ? make_float2(-V4.z, -V4.w) : make_float2(-V4.x, -V4.y);
+                    const float2 t = __ffma2_rn(make_float2(b0, b1), l2e, nl);
+                    const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
+                    float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+                    bool ok0 = true, ok1 = true;
+                    if (!full) {
+                        const int l0 = h2 ? lo4.z : lo4.x, l1 = h2 ? lo4.w : lo4.y;
+                        const int u0 = h2 ? hi4.z : hi4.x, u1 = h2 ? hi4.w : hi4.y;
+                        ok0 = j >= l0 && j <= u0;
+                        ok1 = j >= l1 && j <= u1;
+                        pr.x = ok0 ? pr.x : 0.f;
+                        pr.y = ok1 ? pr.y : 0.f;
+                    }
+                    const float2 ds =
+                        __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv));
+                    if (ok0 && (all_in_extent || c - r < extent_left)) dst0[size_t(c) * dstride] = ds.x;
+                    if (ok1 && (all_in_extent || c + 1 - r < extent_left)) dst0[size_t(c + 1) * dstride] = ds.y;
+                    pk[c >> 1] = pack_bf16x2(pr.x, pr.y);
+                    dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
+                }
             }
             tmem_st16(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
             tmem_st16(tmem + lane_base + L::s_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
@@ -388,7 +423,7 @@ cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUten
     const int nkt = (p.Skv + BK - 1) / BK;
     const long long grid = (long long)nkt * p.B * p.Hkv;
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(320), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nkt);
+    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nkt);
     return cudaGetLastError();
 }
 
@@ -430,7 +465,7 @@ struct Layout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const AttnParams p, const int num_qtiles) {
@@ -507,6 +542,11 @@ __global__ void __launch_bounds__(320, 1)
     auto v_smem = [&](int st, int kb) { return smem + L::V_OFF + (st * KB + kb) * KTILE; };
     auto key0 = [&](int n) { return i0g + BN - (t_begin + n) * BN; };
 
+    // Launched with 384 x 168 registers; warpgroup 2 (producer, MMA issuer, two idle
+    // warps) gives its share to the two elementwise warpgroups
+    // (128 x 40 + 256 x 232 = 384 x 168). Each change sits at the top of its branch.
+    if (warp >= 8) {
+        setmaxnreg_dec<40>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -585,7 +625,9 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
         }
+    }
     } else {
+        setmaxnreg_inc<232>();
         const int w = warp >> 2;
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
@@ -648,26 +690,29 @@ __global__ void __launch_bounds__(320, 1)
             }
             // the row's band buffer is free: prefetch the window of this warpgroup's next step
             if (n + 2 < n_steps && band_needed(n + 2)) issue_band(n + 2);
+            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 l2e = make_float2(kLog2e, kLog2e);
+            const float2 nl2 = make_float2(-lse2, -lse2);
+            const float2 nv2 = make_float2(-dvr, -dvr);
+            const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
             uint32_t dk[32];
 #pragma unroll
             for (int pp = 0; pp < 32; ++pp) {
                 const int c = 2 * pp;
-                float b0 = 0.f, b1 = 0.f;
+                float2 t = nl2;
                 if (use_band) {
                     const uint32_t v = funnel_r(wv[31 - pp], wv[32 - pp], fshift);
-                    b1 = bf16lo_to_f32(v);
-                    b0 = bf16hi_to_f32(v);
+                    t = __ffma2_rn(make_float2(bf16hi_to_f32(v), bf16lo_to_f32(v)), l2e, nl2);
                 }
-                float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, fmaf(b0, kLog2e, -lse2)));
-                float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, fmaf(b1, kLog2e, -lse2)));
+                const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
+                float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
                 if (need_mask) {
-                    const int jj = jk + c;
-                    p0 = (jj >= rb.x && jj <= rb.y) ? p0 : 0.f;
-                    p1 = (jj + 1 >= rb.x && jj + 1 <= rb.y) ? p1 : 0.f;
+                    pr.x = (c >= c_lo && c <= c_hi) ? pr.x : 0.f;
+                    pr.y = (c + 1 >= c_lo && c + 1 <= c_hi) ? pr.y : 0.f;
                 }
-                const float d0v = p0 * (__uint_as_float(dp[c]) - dvr);
-                const float d1v = p1 * (__uint_as_float(dp[c + 1]) - dvr);
-                dk[pp] = pack_bf16x2(d0v, d1v);
+                const float2 ds =
+                    __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv2));
+                dk[pp] = pack_bf16x2(ds.x, ds.y);
             }
             tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
             tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
@@ -730,7 +775,7 @@ cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUten
     const int nqt = (p.S + BM - 1) / BM;
     const long long grid = (long long)nqt * p.B * p.Hq;
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(320), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nqt);
+    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nqt);
     return cudaGetLastError();
 }
 

@@ -60,7 +60,9 @@ struct Layout {
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
-    static constexpr int NWARPS = 4 * NH + 2;
+    // NH = 2: three full warpgroups (softmax A, softmax B, producer + MMA + 2
+    // idle warps) so that registers can be moved between warpgroups.
+    static constexpr int NWARPS = (NH == 2) ? 12 : 6;
     static constexpr uint32_t TMEM_COLS = (NH * (128 + D) <= 256) ? 256u : 512u;
     static constexpr uint32_t s_col(int s) { return uint32_t(s * 128); }
     static constexpr uint32_t o_col(int s) { return uint32_t(NH * 128 + s * D); }
@@ -70,7 +72,7 @@ __device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return -floor_div(-a, b); }
 
 template <int D, int NH>
-__global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
+__global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const int num_qtiles) {
     using L = Layout<D, NH>;
@@ -152,6 +154,11 @@ __global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
     auto k_smem = [&](int kb) { return smem + L::K_OFF + kb * TILE_BYTES; };
     auto v_smem = [&](int kb) { return smem + L::V_OFF + kb * TILE_BYTES; };
 
+    // With NH = 2 the kernel is launched with 384 x 168 registers and the producer
+    // warpgroup gives its share to the two softmax warpgroups (128 x 40 + 256 x 232
+    // = 384 x 168). Each budget change sits at the top of its role's branch.
+    if (warp >= 4 * NH) {
+        if constexpr (NH == 2) setmaxnreg_dec<40>();
     if (warp == TMA_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && n_steps > 0) {
@@ -236,7 +243,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
         }
+    }
     } else {
+        if constexpr (NH == 2) setmaxnreg_inc<232>();
         // ------------------------------------------------------------ softmax
         const int s = warp >> 2;
         const int wq = warp & 3;
@@ -250,7 +259,6 @@ __global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
         const float sigma = row_in ? p.sink[(size_t(b) * p.S + i) * p.Hq + h] : 0.f;
         float m2 = sigma * kLog2e;  // lazily rescaled running maximum, log2 units
         float l = 1.f;              // running denominator; the sink contributes exp(0)
-        float l_r = 1.f;            // same, over BF16-rounded probabilities
 
         uint8_t* band = smem + L::BAND_OFF + s * BAND_BYTES;
         const int unit = band_unit(r);
@@ -293,74 +301,96 @@ __global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
             tmem_ld32(tmem + lane_base + L::s_col(s) + 64, *reinterpret_cast<uint32_t(*)[32]>(&x[64]));
             tmem_ld32(tmem + lane_base + L::s_col(s) + 96, *reinterpret_cast<uint32_t(*)[32]>(&x[96]));
             tmem_wait_ld();
-            if (use_band) cp_async_wait_all();
 
-            // pass 1: logits (natural units) and the row maximum
-            float mx = -INFINITY;
+            // pass 1: the row maximum, in the units of `coef` (which turns x into log2 units)
+            float mx, coef;
+            if (!use_band && !need_mask) {
+                // no relative logit and no mask in this step: x stays the raw score and,
+                // since scale > 0, max(scale * s) = scale * max(s)
+                float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t w[17];
-                if (use_band) {
-#pragma unroll
-                    for (int q = 0; q < 17; ++q) w[q] = band_words[g_r + 48 - 16 * c4 + q];
+                for (int c = 0; c < 128; c += 8) {
+                    a0 = fmax3(a0, __uint_as_float(x[c + 0]), __uint_as_float(x[c + 1]));
+                    a1 = fmax3(a1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+                    a2 = fmax3(a2, __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+                    a3 = fmax3(a3, __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
                 }
+                mx = fmax3(a0, a1, fmaxf(a2, a3));
+                coef = p.scale_log2;
+            } else {
+                // x becomes the logit scale * s + profile bias (natural units), masked
+                if (use_band) cp_async_wait_all();
+                const int c_lo = rb.x - j0, c_hi = rb.y - j0;  // allowed columns of this row
+                const float2 sc2 = make_float2(p.scale, p.scale);
+                float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-                for (int pp = 0; pp < 16; ++pp) {
-                    const int c = 32 * c4 + 2 * pp;
-                    float b0 = 0.f, b1 = 0.f;
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t w[17];
                     if (use_band) {
-                        const uint32_t v = funnel_r(w[15 - pp], w[16 - pp], fshift);
-                        b1 = bf16lo_to_f32(v);  // column c+1
-                        b0 = bf16hi_to_f32(v);  // column c
+#pragma unroll
+                        for (int q = 0; q < 17; ++q) w[q] = band_words[g_r + 48 - 16 * c4 + q];
                     }
-                    float y0 = fmaf(__uint_as_float(x[c]), p.scale, b0);
-                    float y1 = fmaf(__uint_as_float(x[c + 1]), p.scale, b1);
-                    if (need_mask) {
-                        const int j = j0 + c;
-                        y0 = (j >= rb.x && j <= rb.y) ? y0 : -INFINITY;
-                        y1 = (j + 1 >= rb.x && j + 1 <= rb.y) ? y1 : -INFINITY;
+#pragma unroll
+                    for (int pp = 0; pp < 16; ++pp) {
+                        const int c = 32 * c4 + 2 * pp;
+                        float2 bias = make_float2(0.f, 0.f);
+                        if (use_band) {
+                            const uint32_t v = funnel_r(w[15 - pp], w[16 - pp], fshift);
+                            bias.x = bf16hi_to_f32(v);  // column c
+                            bias.y = bf16lo_to_f32(v);  // column c+1
+                        }
+                        float2 y = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2,
+                                              bias);
+                        if (need_mask) {
+                            y.x = (c >= c_lo && c <= c_hi) ? y.x : -INFINITY;
+                            y.y = (c + 1 >= c_lo && c + 1 <= c_hi) ? y.y : -INFINITY;
+                        }
+                        x[c] = __float_as_uint(y.x);
+                        x[c + 1] = __float_as_uint(y.y);
+                        if (pp & 1)
+                            a1 = fmax3(a1, y.x, y.y);
+                        else
+                            a0 = fmax3(a0, y.x, y.y);
                     }
-                    x[c] = __float_as_uint(y0);
-                    x[c + 1] = __float_as_uint(y1);
-                    mx = fmaxf(mx, fmaxf(y0, y1));
                 }
+                mx = fmaxf(a0, a1);
+                coef = kLog2e;
+                // this row's band buffer is free again: prefetch the next step's window
+                // (band_needed is non-increasing in n, so only this path can need it)
+                if (n + 1 < n_steps && band_needed(n + 1)) issue_band(n + 1);
             }
-            // the band buffer of this row is free again: prefetch the next step's window
-            if (n + 1 < n_steps && band_needed(n + 1)) issue_band(n + 1);
 
-            // lazy maximum update (log2 units)
-            const float mx2 = mx * kLog2e;
-            const bool bump = mx2 > m2 + kRescaleThreshold;
+            // running maximum (log2 units): exact on the first step, lazily moved after
+            const float mx2 = mx * coef;
+            const bool bump = (n == 0) ? (mx2 > m2) : (mx2 > m2 + kRescaleThreshold);
             float alpha = 1.f;
             if (bump) {
                 alpha = ex2_approx(m2 - mx2);
                 l *= alpha;
-                l_r *= alpha;
                 m2 = mx2;
             }
             const float base = (m2 == -INFINITY) ? 0.f : m2;
 
-            // pass 2: probabilities, BF16 pack, row sum, store P over the S columns
-            float rowsum = 0.f, rowsum_r = 0.f;
+            // pass 2: probabilities, row sum, BF16 pack, store P over the S columns
+            const float2 c2 = make_float2(coef, coef), nb2 = make_float2(-base, -base);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int c = 32 * q + 2 * u;
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(x[c]), kLog2e, -base));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(x[c + 1]), kLog2e, -base));
-                    pk[u] = pack_bf16x2(p0, p1);
-                    rowsum += p0 + p1;
-                    // the output is normalised by the sum of the BF16-rounded
-                    // probabilities that the PV product uses (numerator and denominator
-                    // share the rounding); lse uses the exact sum
-                    rowsum_r += bf16lo_to_f32(pk[u]) + bf16hi_to_f32(pk[u]);
+                    const float2 t = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), c2, nb2);
+                    const float2 pr = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    pk[u] = pack_bf16x2(pr.x, pr.y);
+                    if (u & 1)
+                        acc1 = __fadd2_rn(acc1, pr);
+                    else
+                        acc0 = __fadd2_rn(acc0, pr);
                 }
                 tmem_st16(tmem + lane_base + L::s_col(s) + 16 * q, pk);
             }
-            l += rowsum;
-            l_r += rowsum_r;
+            l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
 
             // rescale O when a row of this warp moved its maximum (O of step n-1 is complete:
             // the S MMA of this step was committed after it)
@@ -388,7 +418,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 2), 1)
             tc_fence_after();
         }
         if (ok) {
-            const float inv_l = (l_r > 0.f) ? 1.f / l_r : 0.f;
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             float* orow = p.out + ((size_t(b) * p.S + i) * p.Hq + h) * size_t(D);
             if (n_steps > 0) {
 #pragma unroll 1
