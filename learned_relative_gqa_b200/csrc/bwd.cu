@@ -45,6 +45,7 @@ constexpr int BAND_PITCH = BAND_CHUNKS * 16;
 constexpr int BAND_BYTES = BQ * BAND_PITCH;
 constexpr int KTILE = BK * 128;      // [128 rows x 64 bf16] box
 constexpr int QTILE = BQ * 128;      // [64 rows x 64 bf16] box
+constexpr int NST = 3;               // Q / dO stages (two steps of lookahead)
 
 struct StepInfo {
     int lo[BQ];
@@ -59,12 +60,12 @@ struct Layout {
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = K_OFF + KB * KTILE;
     static constexpr int Q_OFF = V_OFF + KB * KTILE;             // 2 stages
-    static constexpr int DO_OFF = Q_OFF + 2 * KB * QTILE;        // 2 stages
-    static constexpr int BAND_OFF = DO_OFF + 2 * KB * QTILE;     // 2 buffers (one per warpgroup)
+    static constexpr int DO_OFF = Q_OFF + NST * KB * QTILE;      // NST stages
+    static constexpr int BAND_OFF = DO_OFF + NST * KB * QTILE;   // 2 buffers (one per warpgroup)
     static constexpr int INFO_OFF = BAND_OFF + 2 * BAND_BYTES;   // 2 StepInfo
     static constexpr int BAR_OFF = INFO_OFF + 2 * int(sizeof(StepInfo));
-    // kv_full, qd_full[2], qd_empty[2], s_full[2], p_full[2], acc_full, drain
-    static constexpr int NBARS = 11;
+    // kv_full, qd_full[NST], qd_empty[NST], s_full[2], p_full[2], acc_full, drain
+    static constexpr int NBARS = 7 + 2 * NST;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -87,12 +88,12 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* kv_full = bars + 0;
-    uint64_t* qd_full = bars + 1;   // [2]
-    uint64_t* qd_empty = bars + 3;  // [2]
-    uint64_t* s_full = bars + 5;    // [2]
-    uint64_t* p_full = bars + 7;    // [2]
-    uint64_t* acc_full = bars + 9;
-    uint64_t* drain = bars + 10;
+    uint64_t* qd_full = bars + 1;              // [NST]
+    uint64_t* qd_empty = bars + 1 + NST;       // [NST]
+    uint64_t* s_full = bars + 1 + 2 * NST;     // [2]
+    uint64_t* p_full = bars + 3 + 2 * NST;     // [2]
+    uint64_t* acc_full = bars + 5 + 2 * NST;
+    uint64_t* drain = bars + 6 + 2 * NST;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -107,9 +108,11 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NST; ++u) {
             mbar_init(&qd_full[u], 1);
             mbar_init(&qd_empty[u], 1);
+        }
+        for (int u = 0; u < 2; ++u) {
             mbar_init(&s_full[u], 1);
             mbar_init(&p_full[u], 4);
         }
@@ -166,8 +169,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             int last = -1;
             for (int n = 0; n < n_steps; ++n) {
-                const int st = n & 1;
-                if (!mbar_wait(&qd_empty[st], ((n >> 1) & 1) ^ 1, ctl, p.err, kErrDkdvQFree, p.timeout_ns)) break;
+                const int st = n % NST;
+                if (!mbar_wait(&qd_empty[st], ((n / NST) & 1) ^ 1, ctl, p.err, kErrDkdvQFree, p.timeout_ns)) break;
                 const int h = step_h(n), i0 = step_qt(n) * BQ;
                 mbar_arrive_expect_tx(&qd_full[st], 2 * KB * QTILE);
                 for (int kb = 0; kb < KB; ++kb) {
@@ -177,15 +180,15 @@ __global__ void __launch_bounds__(384, 1)
                 last = n;
             }
             mbar_wait_drain(kv_full, 0, p.timeout_ns);
-            for (int n = (last > 0 ? last - 1 : 0); n <= last; ++n)
-                if (n >= 0) mbar_wait_drain(&qd_full[n & 1], (n >> 1) & 1, p.timeout_ns);
+            for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
+                mbar_wait_drain(&qd_full[n % NST], (n / NST) & 1, p.timeout_ns);
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BQ, 0, 0);
             constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
             auto issue_sdp = [&](int n) {
-                const int st = n & 1, bb = n & 1;
+                const int st = n % NST, bb = n & 1;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int kb = kk >> 2, kin = kk & 3;
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             for (int n = 0; ok && n < n_steps; ++n) {
                 if (n + 1 < n_steps) {
-                    ok = mbar_wait(&qd_full[(n + 1) & 1], ((n + 1) >> 1) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns);
+                    ok = mbar_wait(&qd_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns);
                     if (!ok) break;
                     tc_fence_after();
                     issue_sdp(n + 1);
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(384, 1)
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDkdvP, p.timeout_ns);
                 if (!ok) break;
                 tc_fence_after();
-                const int st = n & 1, bb = n & 1;
+                const int st = n % NST, bb = n & 1;
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {
                     const uint64_t bdo = sdesc_sw128(smem_u32(do_smem(st, 0)) + kk * 2048, QTILE, 1024);
@@ -441,6 +444,7 @@ constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
 constexpr int BAND_BYTES = BAND_UNITS * 16;
 constexpr int QTILE = BM * 128;       // [128 x 64 bf16]
 constexpr int KTILE = BN * 128;       // [64 x 64 bf16]
+constexpr int NST = 3;                // K / V stages (two steps of lookahead)
 
 __host__ __device__ constexpr int band_unit(int r) { return BAND_CHUNKS * r + 2 * (r >> 3); }
 
@@ -449,12 +453,12 @@ struct Layout {
     static constexpr int KB = D / 64;
     static constexpr int Q_OFF = 0;
     static constexpr int DO_OFF = Q_OFF + KB * QTILE;
-    static constexpr int K_OFF = DO_OFF + KB * QTILE;        // 2 stages
-    static constexpr int V_OFF = K_OFF + 2 * KB * KTILE;     // 2 stages
-    static constexpr int BAND_OFF = V_OFF + 2 * KB * KTILE;  // 2 buffers (one per warpgroup)
+    static constexpr int K_OFF = DO_OFF + KB * QTILE;          // NST stages
+    static constexpr int V_OFF = K_OFF + NST * KB * KTILE;     // NST stages
+    static constexpr int BAND_OFF = V_OFF + NST * KB * KTILE;  // 2 buffers (one per warpgroup)
     static constexpr int BAR_OFF = BAND_OFF + 2 * BAND_BYTES;
-    // q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], acc_full, drain
-    static constexpr int NBARS = 11;
+    // q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], acc_full, drain
+    static constexpr int NBARS = 7 + 2 * NST;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -476,12 +480,12 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
-    uint64_t* kv_full = bars + 1;   // [2]
-    uint64_t* kv_empty = bars + 3;  // [2]
-    uint64_t* s_full = bars + 5;    // [2]
-    uint64_t* p_full = bars + 7;    // [2]
-    uint64_t* acc_full = bars + 9;
-    uint64_t* drain = bars + 10;
+    uint64_t* kv_full = bars + 1;              // [NST]
+    uint64_t* kv_empty = bars + 1 + NST;       // [NST]
+    uint64_t* s_full = bars + 1 + 2 * NST;     // [2]
+    uint64_t* p_full = bars + 3 + 2 * NST;     // [2]
+    uint64_t* acc_full = bars + 5 + 2 * NST;
+    uint64_t* drain = bars + 6 + 2 * NST;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -498,9 +502,11 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NST; ++u) {
             mbar_init(&kv_full[u], 1);
             mbar_init(&kv_empty[u], 1);
+        }
+        for (int u = 0; u < 2; ++u) {
             mbar_init(&s_full[u], 1);
             mbar_init(&p_full[u], 4);
         }
@@ -560,8 +566,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             int last = -1;
             for (int n = 0; n < n_steps; ++n) {
-                const int st = n & 1;
-                if (!mbar_wait(&kv_empty[st], ((n >> 1) & 1) ^ 1, ctl, p.err, kErrDqKVFree, p.timeout_ns)) break;
+                const int st = n % NST;
+                if (!mbar_wait(&kv_empty[st], ((n / NST) & 1) ^ 1, ctl, p.err, kErrDqKVFree, p.timeout_ns)) break;
                 const int jk = key0(n);
                 mbar_arrive_expect_tx(&kv_full[st], 2 * KB * KTILE);
                 for (int kb = 0; kb < KB; ++kb) {
@@ -571,15 +577,15 @@ __global__ void __launch_bounds__(384, 1)
                 last = n;
             }
             mbar_wait_drain(q_full, 0, p.timeout_ns);
-            for (int n = (last > 0 ? last - 1 : 0); n <= last; ++n)
-                if (n >= 0) mbar_wait_drain(&kv_full[n & 1], (n >> 1) & 1, p.timeout_ns);
+            for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
+                mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.timeout_ns);
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
             constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);
             auto issue_sdp = [&](int n) {
-                const int st = n & 1, bb = n & 1;
+                const int st = n % NST, bb = n & 1;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int kb = kk >> 2, kin = kk & 3;
@@ -604,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             for (int n = 0; ok && n < n_steps; ++n) {
                 if (n + 1 < n_steps) {
-                    ok = mbar_wait(&kv_full[(n + 1) & 1], ((n + 1) >> 1) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
+                    ok = mbar_wait(&kv_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
                     if (!ok) break;
                     tc_fence_after();
                     issue_sdp(n + 1);
@@ -612,7 +618,7 @@ __global__ void __launch_bounds__(384, 1)
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
                 if (!ok) break;
                 tc_fence_after();
-                const int st = n & 1, bb = n & 1;
+                const int st = n % NST, bb = n & 1;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, 0)) + kk * 2048, KTILE, 1024);
