@@ -34,25 +34,28 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out_path: str = LIB_PATH, defines: tuple = ()) -> str:
+    """Compile the library. ``defines`` / ``out_path`` build diagnostic variants
+    (for example ``INKLING_TRACE``) next to, not over, the product library."""
+    if not force and not defines and out_path == LIB_PATH and not _stale():
         return LIB_PATH
     objs = []
-    build_dir = os.path.join(ROOT, "_build")
+    build_dir = os.path.join(ROOT, "_build", "-".join(defines) or "default")
     os.makedirs(build_dir, exist_ok=True)
     common = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INCLUDE,
               "--expt-relaxed-constexpr"]
     if verbose:
         common += ["-Xptxas", "-v"]
+    common += [f"-D{d}" for d in defines]
     for src in SOURCES:
         obj = os.path.join(build_dir, src.replace(".cu", ".o"))
         cmd = common + ["-c", os.path.join(CSRC, src), "-o", obj]
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB_PATH + ".tmp"
+    tmp = out_path + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, out_path)
+    return out_path
 
 
 if __name__ == "__main__":

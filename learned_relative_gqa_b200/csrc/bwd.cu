@@ -85,7 +85,9 @@ __global__ void __launch_bounds__(384, 1)
     constexpr int KB = L::KB;
     constexpr int TMA_WARP = 8, MMA_WARP = 9;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
+    // knowing that every pointer derived from it addresses shared memory
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* kv_full = bars + 0;
     uint64_t* qd_full = bars + 1;              // [NST]
@@ -177,6 +179,7 @@ __global__ void __launch_bounds__(384, 1)
                     tma_load_4d(q_smem(st, kb), &tm_q, &qd_full[st], kb * 64, h, i0, b);
                     tma_load_4d(do_smem(st, kb), &tm_do, &qd_full[st], kb * 64, h, i0, b);
                 }
+                IRA_TRACE(p, 21, n);
                 last = n;
             }
             mbar_wait_drain(kv_full, 0, p.timeout_ns);
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ss(tmem + L::dp_col(bb), av, bd, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[bb]);
+                IRA_TRACE(p, 22, n);
             };
             bool ok = mbar_wait(kv_full, 0, ctl, p.err, kErrDkdvKV, p.timeout_ns) &&
                       mbar_wait(&qd_full[0], 0, ctl, p.err, kErrDkdvQ, p.timeout_ns);
@@ -220,6 +224,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDkdvP, p.timeout_ns);
                 if (!ok) break;
+                IRA_TRACE(p, 23, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
 #pragma unroll
@@ -235,6 +240,7 @@ __global__ void __launch_bounds__(384, 1)
                            (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&qd_empty[st]);
+                IRA_TRACE(p, 24, n);
             }
             if (ok) mma_commit(acc_full);
             mma_commit(drain);
@@ -303,6 +309,7 @@ __global__ void __launch_bounds__(384, 1)
                 ok = false;
                 break;
             }
+            if (tid == 0) IRA_TRACE(p, 25 + 3 * w, n);
             tc_fence_after();
             uint32_t sv[64], dp[64];
             tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -310,6 +317,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld32(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
             tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
             tmem_wait_ld();
+            if (tid == 0) IRA_TRACE(p, 31, n);
 
             // Band reads. Column cc reads element (m_cc + 127 - r) of band row cc, where
             // m_cc = (delta + cc - 127) mod 8 repeats every 8 columns: eight per-step
@@ -319,60 +327,67 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 bptr[u] = reinterpret_cast<const uint16_t*>(band + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r));
-            // dprofiles[b, h, i0 + c, delta + c - r] lives at dst0 + c * (R + 1)
-            float* dst0 = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) + (delta - r);
+            // dprofiles[b, h, i0 + c, delta + c - r] for column c: one pointer stepped by R + 1
+            float* dptr = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) + (delta - r);
             const size_t dstride = size_t(p.R) + 1;
-            const bool all_in_extent = delta + BQ - 1 < p.R;  // every distance of the step is < R
-            const int extent_left = p.R - delta;               // d < R  <=>  c - r < extent_left
-            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-            const float2 l2e = make_float2(kLog2e, kLog2e);
+            // d = delta + c - r < R  <=>  c < R - delta + r  (no limit when the whole step is inside R)
+            const int c_lim = (delta + BQ - 1 < p.R) ? BQ : p.R - delta + r;
+            const float* lse2v = info->lse2;
+            const float* dvv = info->dv;
             uint32_t pk[32], dk[32];
 #pragma unroll
-            for (int c4 = 0; c4 < BQ / 4; ++c4) {
-                const float4 L4 = reinterpret_cast<const float4*>(info->lse2)[c4];  // broadcast reads
-                const float4 V4 = reinterpret_cast<const float4*>(info->dv)[c4];
-                int4 lo4 = make_int4(0, 0, 0, 0), hi4 = make_int4(0, 0, 0, 0);
-                if (!full) {
-                    lo4 = reinterpret_cast<const int4*>(info->lo)[c4];
-                    hi4 = reinterpret_cast<const int4*>(info->hi)[c4];
+            for (int c16 = 0; c16 < BQ / 16; ++c16) {
+                // loads of this 16-column chunk, issued together
+                float lse_c[16], dv_c[16], bias_c[16];
+                int lo_c[16], hi_c[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int c = 16 * c16 + u;
+                    lse_c[u] = lse2v[c];
+                    dv_c[u] = dvv[c];
+                    bias_c[u] = __uint_as_float(uint32_t(bptr[c & 7][1088 * (c >> 3)]) << 16);
+                    if (!full) {
+                        lo_c[u] = info->lo[c];
+                        hi_c[u] = info->hi[c];
+                    }
                 }
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int c = 4 * c4 + 2 * h2;
-                    const float b0 = __uint_as_float(uint32_t(bptr[c & 7][1088 * (c >> 3)]) << 16);
-                    const float b1 = __uint_as_float(uint32_t(bptr[(c + 1) & 7][1088 * ((c + 1) >> 3)]) << 16);
-                    const float2 nl = h2 ? make_float2(-L4.z, -L4.w) : make_float2(-L4.x, -L4.y);
-                    const float2 nv = h2 ? make_float2(-V4.z, -V4.w) : make_float2(-V4.x, -V4.y);
-                    const float2 t = __ffma2_rn(make_float2(b0, b1), l2e, nl);
-                    const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
-                    float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
-                    bool ok0 = true, ok1 = true;
-                    if (!full) {
-                        const int l0 = h2 ? lo4.z : lo4.x, l1 = h2 ? lo4.w : lo4.y;
-                        const int u0 = h2 ? hi4.z : hi4.x, u1 = h2 ? hi4.w : hi4.y;
-                        ok0 = j >= l0 && j <= u0;
-                        ok1 = j >= l1 && j <= u1;
-                        pr.x = ok0 ? pr.x : 0.f;
-                        pr.y = ok1 ? pr.y : 0.f;
+                for (int u = 0; u < 16; u += 2) {
+                    const int c = 16 * c16 + u;
+                    float pr[2], ds[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float t = fmaf(bias_c[u + e], kLog2e, -lse_c[u + e]);
+                        float pv = ex2_approx(fmaf(__uint_as_float(sv[c + e]), p.scale_log2, t));
+                        bool ok = true;
+                        if (!full) {
+                            ok = j >= lo_c[u + e] && j <= hi_c[u + e];
+                            pv = ok ? pv : 0.f;
+                        }
+                        const float dsv = pv * (__uint_as_float(dp[c + e]) - dv_c[u + e]);
+                        if (ok && c + e < c_lim) __stcs(dptr, dsv);
+                        dptr += dstride;
+                        pr[e] = pv;
+                        ds[e] = dsv;
                     }
-                    const float2 ds =
-                        __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv));
-                    if (ok0 && (all_in_extent || c - r < extent_left)) dst0[size_t(c) * dstride] = ds.x;
-                    if (ok1 && (all_in_extent || c + 1 - r < extent_left)) dst0[size_t(c + 1) * dstride] = ds.y;
-                    pk[c >> 1] = pack_bf16x2(pr.x, pr.y);
-                    dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
+                    pk[c >> 1] = pack_bf16x2(pr[0], pr[1]);
+                    dk[c >> 1] = pack_bf16x2(ds[0], ds[1]);
                 }
             }
+            if (tid == 0) IRA_TRACE(p, 32, n);
             tmem_st16(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
             tmem_st16(tmem + lane_base + L::s_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
             tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
             tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
             tmem_wait_st();
+            if (tid == 0) IRA_TRACE(p, 33, n);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[bb]);
+            if (tid == 0) IRA_TRACE(p, 26 + 3 * w, n);
             named_bar_sync(1 + w, 128);  // band and info of this step fully consumed
             if (n + 2 < n_steps) stage(n + 2);
+            if (tid == 0) IRA_TRACE(p, 27 + 3 * w, n);
         }
         cp_async_wait_all();
 
@@ -477,7 +492,9 @@ __global__ void __launch_bounds__(384, 1)
     constexpr int KB = L::KB;
     constexpr int TMA_WARP = 8, MMA_WARP = 9;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
+    // knowing that every pointer derived from it addresses shared memory
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
     uint64_t* kv_full = bars + 1;              // [NST]
@@ -574,6 +591,7 @@ __global__ void __launch_bounds__(384, 1)
                     tma_load_4d(k_smem(st, kb), &tm_k, &kv_full[st], kb * 64, g, jk, b);
                     tma_load_4d(v_smem(st, kb), &tm_v, &kv_full[st], kb * 64, g, jk, b);
                 }
+                IRA_TRACE(p, 41, n);
                 last = n;
             }
             mbar_wait_drain(q_full, 0, p.timeout_ns);
@@ -601,6 +619,7 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ss(tmem + L::dp_col(bb), ad, bv, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[bb]);
+                IRA_TRACE(p, 42, n);
             };
             bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns) &&
                       mbar_wait(&kv_full[0], 0, ctl, p.err, kErrDqKV, p.timeout_ns);
@@ -617,6 +636,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
                 if (!ok) break;
+                IRA_TRACE(p, 43, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
 #pragma unroll
@@ -626,6 +646,7 @@ __global__ void __launch_bounds__(384, 1)
                            (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&kv_empty[st]);
+                IRA_TRACE(p, 44, n);
             }
             if (ok) mma_commit(acc_full);
             mma_commit(drain);
@@ -681,6 +702,7 @@ __global__ void __launch_bounds__(384, 1)
                 ok = false;
                 break;
             }
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 45 + 2 * w, n);
             tc_fence_after();
             uint32_t sv[64], dp[64];
             tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -726,6 +748,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[bb]);
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 46 + 2 * w, n);
         }
         cp_async_wait_all();
 

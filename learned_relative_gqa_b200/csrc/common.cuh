@@ -102,6 +102,9 @@ struct AttnParams {
     float* dk;
     float* dv;
     float* dprofiles;
+    // pipeline timeline of one CTA (only in builds with INKLING_TRACE; null otherwise)
+    unsigned long long* trace;
+    int trace_cta;
 };
 
 }  // namespace ira

@@ -80,7 +80,9 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
     constexpr int TMA_WARP = 4 * NH, MMA_WARP = 4 * NH + 1;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
+    // knowing that every pointer derived from it addresses shared memory
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
     uint64_t* k_full = bars + 1;
@@ -174,10 +176,12 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                 if (!mbar_wait(k_empty, (n & 1) ^ 1, ctl, p.err, kErrFwdKFree, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(k_full, KB * TILE_BYTES);
                 for (int kb = 0; kb < KB; ++kb) tma_load_4d(k_smem(kb), &tm_k, k_full, kb * 64, g, j0, b);
+                IRA_TRACE(p, 1, n);
                 nk = n;
                 if (!mbar_wait(v_empty, (n & 1) ^ 1, ctl, p.err, kErrFwdVFree, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(v_full, KB * TILE_BYTES);
                 for (int kb = 0; kb < KB; ++kb) tma_load_4d(v_smem(kb), &tm_v, v_full, kb * 64, g, j0, b);
+                IRA_TRACE(p, 2, n);
                 nv = n;
             }
             // never leave a copy in flight into shared memory of an exiting CTA
@@ -210,29 +214,36 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
             bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns) &&
                       mbar_wait(k_full, 0, ctl, p.err, kErrFwdK, p.timeout_ns);
             if (ok) {
+                IRA_TRACE(p, 9, 0);
                 tc_fence_after();
                 for (int s = 0; s < NH; ++s) {
                     issue_s(s);
                     mma_commit(&s_full[s]);
+                    IRA_TRACE(p, 3 + s, 0);
                 }
                 mma_commit(k_empty);
             }
             for (int n = 0; ok && n < n_steps; ++n) {
                 ok = mbar_wait(v_full, n & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
+                IRA_TRACE(p, 10, n);
                 for (int s = 0; ok && s < NH; ++s) {
                     ok = mbar_wait(&p_full[s], n & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
                     if (!ok) break;
+                    IRA_TRACE(p, 7 + s, n);
                     tc_fence_after();
                     issue_o(s, n > 0);
+                    IRA_TRACE(p, 5 + s, n);
                     if (s == NH - 1) mma_commit(v_empty);
                     if (n + 1 < n_steps) {
                         if (s == 0) {
                             ok = mbar_wait(k_full, (n + 1) & 1, ctl, p.err, kErrFwdK, p.timeout_ns);
                             if (!ok) break;
+                            IRA_TRACE(p, 9, n + 1);
                             tc_fence_after();
                         }
                         issue_s(s);
                         mma_commit(&s_full[s]);
+                        IRA_TRACE(p, 3 + s, n + 1);
                         if (s == NH - 1) mma_commit(k_empty);
                     }
                 }
@@ -294,6 +305,7 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                 ok = false;
                 break;
             }
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 11 + 3 * s, n);
             tc_fence_after();
             uint32_t x[128];
             tmem_ld32(tmem + lane_base + L::s_col(s) + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -360,6 +372,7 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                 if (n + 1 < n_steps && band_needed(n + 1)) issue_band(n + 1);
             }
 
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 12 + 3 * s, n);
             // running maximum (log2 units): exact on the first step, lazily moved after
             const float mx2 = mx * coef;
             const bool bump = (n == 0) ? (mx2 > m2) : (mx2 > m2 + kRescaleThreshold);
@@ -409,6 +422,7 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[s]);
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 13 + 3 * s, n);
         }
         cp_async_wait_all();
 

@@ -64,6 +64,12 @@ cudaError_t note(cudaError_t e) {
     return e;
 }
 
+#ifdef INKLING_TRACE
+// Pipeline timeline of one CTA (diagnostic builds only).
+unsigned long long* g_trace_buf = nullptr;
+int g_trace_cta = 0;
+#endif
+
 // Optional per-launch timing events (inkling_rel_attn_set_timing_events).
 cudaEvent_t const* g_events = nullptr;
 int g_event_pairs = 0;
@@ -160,6 +166,10 @@ AttnParams base_params(const inkling_rel_attn_dims* d, const Ws& w, const uint16
     p.row_bounds = w.row_bounds();
     p.tile_bounds = w.tiles();
     p.err = w.ctl();
+#ifdef INKLING_TRACE
+    p.trace = g_trace_buf;
+    p.trace_cta = g_trace_cta;
+#endif
     return p;
 }
 
@@ -421,6 +431,15 @@ inkling_status inkling_rel_attn_set_timing_events(void* const* events, int n_pai
 const char* inkling_rel_attn_last_cuda_error(void) {
     return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
 }
+
+#ifdef INKLING_TRACE
+// Diagnostic builds only: record the pipeline timeline of CTA `cta` of the next
+// attention kernels into the device buffer `buf` (see ira::trace_event).
+void inkling_rel_attn_debug_trace(void* buf, int cta) {
+    g_trace_buf = static_cast<unsigned long long*>(buf);
+    g_trace_cta = cta;
+}
+#endif
 
 const char* inkling_status_string(inkling_status status) {
     switch (status) {

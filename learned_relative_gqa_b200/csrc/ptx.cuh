@@ -48,6 +48,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Same, but the thread may sleep (not issue) until the phase completes or about
+// kSuspendHintNs pass, so waiting warps leave the issue slots to working warps.
+constexpr uint32_t kSuspendHintNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
 
 // Shared control block of a CTA: `abort` is raised by the first wait that
 // runs out so that every other role stops waiting too.
@@ -64,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, CtaCon
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
         if (globaltimer_ns() - t0 > timeout_ns) {
             atomicExch(&ctl->abort, 1);
@@ -86,7 +99,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, CtaCon
 // Bounded wait used while draining at teardown: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
     return true;
@@ -280,4 +293,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// optional pipeline timeline (compiled only with -DINKLING_TRACE)
+// ---------------------------------------------------------------------------
+// Slot (step * 64 + event) of buf receives the SM clock; only CTA `cta`
+// records, steps >= 8192 are dropped. No atomics, so recording does not stall.
+__device__ __forceinline__ void trace_event(unsigned long long* buf, int cta, int ev, int step) {
+    if (buf != nullptr && int(blockIdx.x) == cta && step < 8192) buf[step * 64 + ev] = clock64();
+}
+
 }  // namespace ira
+
+#ifdef INKLING_TRACE
+#define IRA_TRACE(p, ev, step) ::ira::trace_event((p).trace, (p).trace_cta, (ev), (step))
+#else
+#define IRA_TRACE(p, ev, step) ((void)0)
+#endif
