@@ -341,15 +341,22 @@ __global__ void __launch_bounds__(384, 1)
                 float lse_c[16], dv_c[16], bias_c[16];
                 int lo_c[16], hi_c[16];
 #pragma unroll
+                for (int u4 = 0; u4 < 4; ++u4) {  // 128-bit broadcast reads of four columns
+                    const float4 l4 = reinterpret_cast<const float4*>(lse2v)[4 * c16 + u4];
+                    const float4 v4 = reinterpret_cast<const float4*>(dvv)[4 * c16 + u4];
+                    lse_c[4 * u4 + 0] = l4.x; lse_c[4 * u4 + 1] = l4.y; lse_c[4 * u4 + 2] = l4.z; lse_c[4 * u4 + 3] = l4.w;
+                    dv_c[4 * u4 + 0] = v4.x; dv_c[4 * u4 + 1] = v4.y; dv_c[4 * u4 + 2] = v4.z; dv_c[4 * u4 + 3] = v4.w;
+                    if (!full) {
+                        const int4 a4 = reinterpret_cast<const int4*>(info->lo)[4 * c16 + u4];
+                        const int4 b4 = reinterpret_cast<const int4*>(info->hi)[4 * c16 + u4];
+                        lo_c[4 * u4 + 0] = a4.x; lo_c[4 * u4 + 1] = a4.y; lo_c[4 * u4 + 2] = a4.z; lo_c[4 * u4 + 3] = a4.w;
+                        hi_c[4 * u4 + 0] = b4.x; hi_c[4 * u4 + 1] = b4.y; hi_c[4 * u4 + 2] = b4.z; hi_c[4 * u4 + 3] = b4.w;
+                    }
+                }
+#pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int c = 16 * c16 + u;
-                    lse_c[u] = lse2v[c];
-                    dv_c[u] = dvv[c];
                     bias_c[u] = __uint_as_float(uint32_t(bptr[c & 7][1088 * (c >> 3)]) << 16);
-                    if (!full) {
-                        lo_c[u] = info->lo[c];
-                        hi_c[u] = info->hi[c];
-                    }
                 }
 #pragma unroll
                 for (int u = 0; u < 16; u += 2) {

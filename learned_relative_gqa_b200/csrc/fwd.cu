@@ -1,30 +1,42 @@
 // fwd.cu -- forward kernel of learned-relative grouped-query attention (sm_100a).
 //
 // One CTA handles one 128-row query tile of NH query heads (NH = 2 heads of the
-// same KV group when the group size is even, else 1). The K/V tile of each
-// step is loaded once by TMA and shared by both heads; the two heads ping-pong
-// on the tensor core while the other head's softmax runs:
+// same KV group when the group size is even, else 1). Each step covers 64 keys;
+// its K and V tiles are loaded once by TMA and shared by both heads, K through a
+// three-slot ring and V through a two-slot ring, each fed by its own producer.
 //
 //   warps 0..4*NH-1   softmax, one warpgroup per head (thread = query row =
-//                     TMEM lane); also stage the head's profile band
-//   warp  4*NH        TMA producer: Q (once), K and V tiles
-//   warp  4*NH+1      MMA issuer (one thread): S = Q K^T (SMEM x SMEM -> TMEM),
-//                     O += P V (P from TMEM x V from SMEM -> TMEM)
+//                     TMEM lane); each thread also stages its own row's
+//                     profile window (double buffered, warmed in L2 ahead)
+//   warp  4*NH        TMA producer: Q (once), then the K tiles
+//   warp  4*NH+1      MMA issuer of head A (one thread): S = Q K^T (SMEM x SMEM
+//                     -> TMEM), O += P V (P from TMEM x V from SMEM -> TMEM)
+//   warp  4*NH+2      TMA producer: the V tiles
+//   warp  4*NH+3      MMA issuer of head B (NH = 2)
 //
-// Per KV step the softmax warpgroup reads S from TMEM, adds the learned
-// relative logit profiles[b,h,i,d] (d = i_g - j; distances >= R read zeros),
-// masks the step's boundary tiles, keeps a lazily rescaled running maximum
-// initialised with the sink logit (running sum initialised with exp(0) = 1, so
-// the sink enters the denominator with no value row), writes P as BF16 into
-// the S columns of TMEM and, when its maximum moved, rescales O in TMEM.
+// S is double buffered per head in TMEM, so the MMAs for step n+2 are queued
+// right behind the PV products of step n (P of step n lives in the S buffer it
+// aliases) and a softmax warpgroup rarely waits on the tensor core. Each head
+// has its own issuing thread, so the tensor core is fed by the other head while
+// one issuer waits for its softmax or a tile.
+// TMEM: S_A[2], S_B[2] (64 columns each), O_A, O_B (D each).
 //
-// Key tiles are aligned to the query tile: step t covers keys
-// [i_g0 - 128 t, i_g0 - 128 t + 127], so the distance offset of the step is
-// delta = 128 t and row r needs the profile distances [delta + r - 127,
-// delta + r]. Each softmax thread copies exactly that window of its own
-// profile row (17 x 16 B, cp.async with zero fill outside [0, R)) into a band
-// buffer laid out so that the per-column 32-bit gathers of a warp hit 32
-// distinct shared-memory banks: row r starts at 16-byte unit 17 r + 2 (r / 8).
+// Per step the softmax warpgroup reads S, adds the learned relative logit
+// profiles[b,h,i,d] (d = i_g - j; distances >= R read zeros), masks only the
+// steps that cross a document / window / validity boundary, keeps a running
+// maximum that starts at the sink logit and is exact on the first step and
+// lazily moved afterwards, keeps the running denominator (the sink contributes
+// exp(0) = 1, so it enters with no value row), writes P as BF16 over its S
+// buffer, and rescales O in TMEM in the rare steps whose maximum moved (after
+// the previous PV product is known to be complete).
+//
+// Key steps are aligned to the query tile: step u covers keys
+// [i_g0 + 64 - 64 u, i_g0 + 127 - 64 u], so its distance offset is
+// delta = 64 u - 64 and row r needs the distances [delta + r - 63, delta + r].
+// That window starts (r + 1) mod 8 elements past a 16-byte boundary for every
+// step; each softmax thread copies it (9 x 16 B, cp.async, zero fill outside
+// [0, R)) into a buffer whose rows are permuted so that the per-column 32-bit
+// reads of a warp hit 32 distinct shared-memory banks.
 //
 // Operation and argument conventions follow the NeMo AutoModel page for
 // Inkling2FlexAttention.forward; see include/inkling_rel_attn.h.
@@ -39,45 +51,75 @@ namespace ira {
 namespace fwdk {
 
 constexpr int BM = 128;               // query rows per tile (TMEM lanes)
-constexpr int BN = 128;               // keys per step
-constexpr int BAND_CHUNKS = 17;       // 16-byte chunks per band row (136 bf16)
-constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
-constexpr int BAND_BYTES = BAND_UNITS * 16;
-constexpr int TILE_BYTES = BM * 128;  // one [128 rows x 64 bf16] 128B-swizzled box
+constexpr int BN = 64;                // keys per step
+constexpr int KSLOTS = 3;             // K ring slots (two steps of lookahead)
+constexpr int VSLOTS = 2;             // V ring slots
+constexpr int BAND_CHUNKS = 9;        // 16-byte chunks per band row (72 bf16)
+constexpr int BAND_PITCH = BAND_CHUNKS * 16;
+constexpr int BAND_BYTES = BM * BAND_PITCH;
+constexpr int QBOX = BM * 128;        // [128 rows x 64 bf16] 128B-swizzled box
+constexpr int KBOX = BN * 128;        // [64 rows x 64 bf16] box
 
-__host__ __device__ constexpr int band_unit(int r) { return BAND_CHUNKS * r + 2 * (r >> 3); }
+// Row r = 8a + s is stored in slot 8a + ((s + 2a) mod 8): the slot's 16-byte unit
+// index is then congruent to (s + 2a) mod 8 (the pitch is 9 units), which spreads
+// the 32 rows of a warp over all 32 banks for the column-wise reads below.
+__host__ __device__ constexpr int band_slot(int r) { return (r & ~7) | (((r & 7) + 2 * (r >> 3)) & 7); }
 
 template <int D, int NH>
 struct Layout {
     static constexpr int KB = D / 64;
+    static constexpr int SLOT_BYTES = KB * KBOX;
     static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + NH * KB * TILE_BYTES;
-    static constexpr int V_OFF = K_OFF + KB * TILE_BYTES;
-    static constexpr int BAND_OFF = V_OFF + KB * TILE_BYTES;
-    static constexpr int BAR_OFF = BAND_OFF + NH * BAND_BYTES;
-    // q_full, k_full, k_empty, v_full, v_empty, drain, s_full[NH], p_full[NH], o_full[NH]
-    static constexpr int NBARS = 6 + 3 * NH;
+    static constexpr int K_OFF = Q_OFF + NH * KB * QBOX;
+    static constexpr int V_OFF = K_OFF + KSLOTS * SLOT_BYTES;
+    static constexpr int BAND_OFF = V_OFF + VSLOTS * SLOT_BYTES;
+    static constexpr int BAR_OFF = BAND_OFF + NH * 2 * BAND_BYTES;
+    // q_full, k_full[KSLOTS], k_empty[KSLOTS], v_full[VSLOTS], v_empty[VSLOTS], drain,
+    // s_full[NH][2], p_full[NH][2], o_done[NH], o_full[NH]
+    static constexpr int NBARS = 2 + 2 * KSLOTS + 2 * VSLOTS + 6 * NH;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
-    // NH = 2: three full warpgroups (softmax A, softmax B, producer + MMA + 2
-    // idle warps) so that registers can be moved between warpgroups.
-    static constexpr int NWARPS = (NH == 2) ? 12 : 6;
+    // softmax warpgroup(s), then one warpgroup holding the K producer, the MMA
+    // issuers and the V producer (whole warpgroups, so that with NH = 2
+    // registers can be moved between them)
+    static constexpr int NWARPS = 4 * NH + 4;
     static constexpr uint32_t TMEM_COLS = (NH * (128 + D) <= 256) ? 256u : 512u;
-    static constexpr uint32_t s_col(int s) { return uint32_t(s * 128); }
+    static constexpr uint32_t s_col(int s, int buf) { return uint32_t(s * 128 + buf * 64); }
     static constexpr uint32_t o_col(int s) { return uint32_t(NH * 128 + s * D); }
 };
 
 __device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return -floor_div(-a, b); }
 
+// Load K (or V) tiles 0 .. n_steps-1 of this CTA through a ring of NS slots
+// (lane 0 of the producer warp). Before returning, waits for its own copies in
+// flight so that none lands in the shared memory of an exiting CTA.
+template <int NS, int KB>
+__device__ __forceinline__ void produce_ring(const CUtensorMap* tm, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                             int n_steps, int g, int b, int key_first, CtaControl* ctl,
+                                             const AttnParams& p, int site, int trace_ev) {
+    int last = -1;
+    for (int n = 0; n < n_steps; ++n) {
+        const int slot = n % NS;
+        if (!mbar_wait(&empty[slot], ((n / NS) & 1) ^ 1, ctl, p.err, site, p.timeout_ns)) break;
+        mbar_arrive_expect_tx(&full[slot], KB * KBOX);
+        for (int kb = 0; kb < KB; ++kb)
+            tma_load_4d(ring + (slot * KB + kb) * KBOX, tm, &full[slot], kb * 64, g, key_first - n * BN, b);
+        IRA_TRACE(p, trace_ev, n);
+        last = n;
+    }
+    for (int n = (last >= NS ? last - NS + 1 : 0); n <= last; ++n)
+        mbar_wait_drain(&full[n % NS], (n / NS) & 1, p.timeout_ns);
+}
+
 template <int D, int NH>
-__global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
+__global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const int num_qtiles) {
     using L = Layout<D, NH>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 4 * NH, MMA_WARP = 4 * NH + 1;
+    constexpr int K_WARP = 4 * NH, MMA_WARP = 4 * NH + 1, V_WARP = 4 * NH + 2, MMA_WARP_B = 4 * NH + 3;
 
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
@@ -85,14 +127,15 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;
-    uint64_t* k_empty = bars + 2;
-    uint64_t* v_full = bars + 3;
-    uint64_t* v_empty = bars + 4;
-    uint64_t* drain = bars + 5;
-    uint64_t* s_full = bars + 6;
-    uint64_t* p_full = bars + 6 + NH;
-    uint64_t* o_full = bars + 6 + 2 * NH;
+    uint64_t* k_full = bars + 1;                    // [KSLOTS]
+    uint64_t* k_empty = k_full + KSLOTS;            // [KSLOTS]
+    uint64_t* v_full = k_empty + KSLOTS;            // [VSLOTS]
+    uint64_t* v_empty = v_full + VSLOTS;            // [VSLOTS]
+    uint64_t* drain = v_empty + VSLOTS;
+    uint64_t* s_full = drain + 1;                   // [NH][2]
+    uint64_t* p_full = s_full + 2 * NH;             // [NH][2]
+    uint64_t* o_done = p_full + 2 * NH;             // [NH]
+    uint64_t* o_full = o_done + NH;                 // [NH]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -113,14 +156,22 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        mbar_init(k_full, 1);
-        mbar_init(k_empty, 1);
-        mbar_init(v_full, 1);
-        mbar_init(v_empty, 1);
-        mbar_init(drain, 1);
+        // a K or V slot is free once the MMAs of every head's issuer have read it
+        for (int u = 0; u < KSLOTS; ++u) {
+            mbar_init(&k_full[u], 1);
+            mbar_init(&k_empty[u], NH);
+        }
+        for (int u = 0; u < VSLOTS; ++u) {
+            mbar_init(&v_full[u], 1);
+            mbar_init(&v_empty[u], NH);
+        }
+        mbar_init(drain, NH);
         for (int s = 0; s < NH; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 4);
+            mbar_init(&s_full[2 * s + 0], 1);
+            mbar_init(&s_full[2 * s + 1], 1);
+            mbar_init(&p_full[2 * s + 0], 4);
+            mbar_init(&p_full[2 * s + 1], 4);
+            mbar_init(&o_done[s], 1);
             mbar_init(&o_full[s], 1);
         }
         ctl->abort = 0;
@@ -131,13 +182,14 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
             max_hi = max(max_hi, tb[1].max_hi);
             ne += tb[1].n_nonempty;
         }
-        int t_begin = 0, n_steps = 0;
+        int u_begin = 0, n_steps = 0;
         if (ne > 0) {
-            t_begin = max(0, ceil_div_i(i0g - max_hi, BN));
-            const int t_end = floor_div(i0g + BM - 1 - min_lo, BN);
-            n_steps = max(0, t_end - t_begin + 1);
+            // step u covers keys [i0g + 64 - 64 u, i0g + 127 - 64 u]
+            u_begin = max(0, ceil_div_i(i0g + BN - max_hi, BN));
+            const int u_end = floor_div(i0g + 2 * BN - 1 - min_lo, BN);
+            n_steps = max(0, u_end - u_begin + 1);
         }
-        tinfo[0] = t_begin;
+        tinfo[0] = u_begin;
         tinfo[1] = n_steps;
         fence_mbar_init();
     }
@@ -149,114 +201,110 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int t_begin = tinfo[0];
+    const int u_begin = tinfo[0];
     const int n_steps = tinfo[1];
 
-    auto q_smem = [&](int s, int kb) { return smem + L::Q_OFF + (s * KB + kb) * TILE_BYTES; };
-    auto k_smem = [&](int kb) { return smem + L::K_OFF + kb * TILE_BYTES; };
-    auto v_smem = [&](int kb) { return smem + L::V_OFF + kb * TILE_BYTES; };
+    auto q_smem = [&](int s, int kb) { return smem + L::Q_OFF + (s * KB + kb) * QBOX; };
+    auto key0 = [&](int n) { return i0g + BN - (u_begin + n) * BN; };
 
     // With NH = 2 the kernel is launched with 384 x 168 registers and the producer
-    // warpgroup gives its share to the two softmax warpgroups (128 x 40 + 256 x 232
-    // = 384 x 168). Each budget change sits at the top of its role's branch.
+    // warpgroup gives part of its share to the two softmax warpgroups (128 x 80 +
+    // 256 x 208 <= 384 x 168). Each budget change sits at the top of its role's branch.
     if (warp >= 4 * NH) {
-        if constexpr (NH == 2) setmaxnreg_dec<40>();
-    if (warp == TMA_WARP) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && n_steps > 0) {
-            prefetch_tensormap(&tm_q);
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
-            mbar_arrive_expect_tx(q_full, NH * KB * TILE_BYTES);
-            for (int s = 0; s < NH; ++s)
-                for (int kb = 0; kb < KB; ++kb) tma_load_4d(q_smem(s, kb), &tm_q, q_full, kb * 64, h0 + s, i0, b);
-            int nk = -1, nv = -1;
-            for (int n = 0; n < n_steps; ++n) {
-                const int j0 = i0g - (t_begin + n) * BN;
-                if (!mbar_wait(k_empty, (n & 1) ^ 1, ctl, p.err, kErrFwdKFree, p.timeout_ns)) break;
-                mbar_arrive_expect_tx(k_full, KB * TILE_BYTES);
-                for (int kb = 0; kb < KB; ++kb) tma_load_4d(k_smem(kb), &tm_k, k_full, kb * 64, g, j0, b);
-                IRA_TRACE(p, 1, n);
-                nk = n;
-                if (!mbar_wait(v_empty, (n & 1) ^ 1, ctl, p.err, kErrFwdVFree, p.timeout_ns)) break;
-                mbar_arrive_expect_tx(v_full, KB * TILE_BYTES);
-                for (int kb = 0; kb < KB; ++kb) tma_load_4d(v_smem(kb), &tm_v, v_full, kb * 64, g, j0, b);
-                IRA_TRACE(p, 2, n);
-                nv = n;
+        if constexpr (NH == 2) setmaxnreg_dec<80>();
+        if (warp == K_WARP) {
+            // -------------------------------------------------------- Q and K producer
+            if (lane == 0 && n_steps > 0) {
+                prefetch_tensormap(&tm_q);
+                prefetch_tensormap(&tm_k);
+                mbar_arrive_expect_tx(q_full, NH * KB * QBOX);
+                for (int s = 0; s < NH; ++s)
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_4d(q_smem(s, kb), &tm_q, q_full, kb * 64, h0 + s, i0, b);
+                produce_ring<KSLOTS, KB>(&tm_k, smem + L::K_OFF, k_full, k_empty, n_steps, g, b, key0(0), ctl, p,
+                                         kErrFwdKFree, 1);
+                mbar_wait_drain(q_full, 0, p.timeout_ns);
             }
-            // never leave a copy in flight into shared memory of an exiting CTA
-            mbar_wait_drain(q_full, 0, p.timeout_ns);
-            if (nk >= 0) mbar_wait_drain(k_full, nk & 1, p.timeout_ns);
-            if (nv >= 0) mbar_wait_drain(v_full, nv & 1, p.timeout_ns);
-        }
-    } else if (warp == MMA_WARP) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_steps > 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
-            auto issue_s = [&](int s) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int kb = kk >> 2, kin = kk & 3;
-                    const uint64_t ad = sdesc_sw128(smem_u32(q_smem(s, kb)) + kin * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(smem_u32(k_smem(kb)) + kin * 32, 16, 1024);
-                    mma_ss(tmem + L::s_col(s), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_o = [&](int s, bool acc) {
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(smem_u32(v_smem(0)) + kk * 2048, TILE_BYTES, 1024);
-                    mma_ts(tmem + L::o_col(s), tmem + L::s_col(s) + kk * 8, bd, IDESC_O,
-                           (acc || kk > 0) ? 1u : 0u);
-                }
-            };
-            bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns) &&
-                      mbar_wait(k_full, 0, ctl, p.err, kErrFwdK, p.timeout_ns);
-            if (ok) {
-                IRA_TRACE(p, 9, 0);
-                tc_fence_after();
-                for (int s = 0; s < NH; ++s) {
-                    issue_s(s);
-                    mma_commit(&s_full[s]);
-                    IRA_TRACE(p, 3 + s, 0);
-                }
-                mma_commit(k_empty);
+        } else if (warp == V_WARP) {
+            // -------------------------------------------------------- V producer
+            if (lane == 0 && n_steps > 0) {
+                prefetch_tensormap(&tm_v);
+                produce_ring<VSLOTS, KB>(&tm_v, smem + L::V_OFF, v_full, v_empty, n_steps, g, b, key0(0), ctl, p,
+                                         kErrFwdVFree, 2);
             }
-            for (int n = 0; ok && n < n_steps; ++n) {
-                ok = mbar_wait(v_full, n & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
-                IRA_TRACE(p, 10, n);
-                for (int s = 0; ok && s < NH; ++s) {
-                    ok = mbar_wait(&p_full[s], n & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
+        } else if (warp == MMA_WARP || (NH == 2 && warp == MMA_WARP_B)) {
+            // -------------------------------------------------------- MMA issuers
+            // One issuing thread per head, so that one head's waits never hold back
+            // the other head's MMAs. Per step n: O_s += P_s(n) V(n), then
+            // S_s(n+2) = Q_s K(n+2)^T into the S buffer that P_s(n) occupied (the
+            // tensor core runs one thread's MMAs in issue order). The K and V slots
+            // are released once both heads' MMAs that read them have completed.
+            const int s = (warp == MMA_WARP) ? 0 : 1;
+            if (lane == 0 && n_steps > 0) {
+                constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
+                constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
+                const uint32_t k_base = smem_u32(smem + L::K_OFF), v_base = smem_u32(smem + L::V_OFF);
+                const uint32_t q_base = smem_u32(q_smem(s, 0));
+                auto wait_k = [&](int n) {
+                    return mbar_wait(&k_full[n % KSLOTS], (n / KSLOTS) & 1, ctl, p.err, kErrFwdK, p.timeout_ns);
+                };
+                auto issue_s = [&](int n) {
+                    const uint32_t kslot = k_base + (n % KSLOTS) * L::SLOT_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * QBOX + (kk & 3) * 32;
+                        const uint64_t ad = sdesc_sw128(q_base + off, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(kslot + (kk >> 2) * KBOX + (kk & 3) * 32, 16, 1024);
+                        mma_ss(tmem + L::s_col(s, n & 1), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[2 * s + (n & 1)]);
+                    IRA_TRACE(p, 3 + s, n);
+                };
+                auto issue_o = [&](int n) {
+                    const uint32_t vslot = v_base + (n % VSLOTS) * L::SLOT_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        const uint64_t bd = sdesc_sw128(vslot + kk * 2048, KBOX, 1024);
+                        mma_ts(tmem + L::o_col(s), tmem + L::s_col(s, n & 1) + kk * 8, bd, IDESC_O,
+                               (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&o_done[s]);
+                    IRA_TRACE(p, 5 + s, n);
+                };
+                bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
+                for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
+                    ok = wait_k(n);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(n);
+                    mma_commit(&k_empty[n % KSLOTS]);
+                }
+                for (int n = 0; ok && n < n_steps; ++n) {
+                    ok = mbar_wait(&v_full[n % VSLOTS], (n / VSLOTS) & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
+                    if (s == 0) IRA_TRACE(p, 10, n);
+                    // one barrier per S buffer: the softmax may already have finished
+                    // step n + 1 (whose S was issued before this wait)
+                    ok = ok && mbar_wait(&p_full[2 * s + (n & 1)], (n >> 1) & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
+                    if (ok && n + 2 < n_steps) ok = wait_k(n + 2);
                     if (!ok) break;
                     IRA_TRACE(p, 7 + s, n);
                     tc_fence_after();
-                    issue_o(s, n > 0);
-                    IRA_TRACE(p, 5 + s, n);
-                    if (s == NH - 1) mma_commit(v_empty);
-                    if (n + 1 < n_steps) {
-                        if (s == 0) {
-                            ok = mbar_wait(k_full, (n + 1) & 1, ctl, p.err, kErrFwdK, p.timeout_ns);
-                            if (!ok) break;
-                            IRA_TRACE(p, 9, n + 1);
-                            tc_fence_after();
-                        }
-                        issue_s(s);
-                        mma_commit(&s_full[s]);
-                        IRA_TRACE(p, 3 + s, n + 1);
-                        if (s == NH - 1) mma_commit(k_empty);
+                    issue_o(n);
+                    mma_commit(&v_empty[n % VSLOTS]);
+                    if (n + 2 < n_steps) {
+                        issue_s(n + 2);
+                        mma_commit(&k_empty[(n + 2) % KSLOTS]);
                     }
                 }
+                // O is final once every PV product has completed
+                if (ok) mma_commit(&o_full[s]);
+                // wait for every MMA of both issuers before TMEM is released
+                mma_commit(drain);
+                mbar_wait_drain(drain, 0, p.timeout_ns);
             }
-            if (ok)
-                for (int s = 0; s < NH; ++s) mma_commit(&o_full[s]);
-            // wait for every issued MMA before TMEM is released
-            mma_commit(drain);
-            mbar_wait_drain(drain, 0, p.timeout_ns);
         }
-    }
     } else {
-        if constexpr (NH == 2) setmaxnreg_inc<232>();
+        if constexpr (NH == 2) setmaxnreg_inc<208>();
         // ------------------------------------------------------------ softmax
         const int s = warp >> 2;
         const int wq = warp & 3;
@@ -268,50 +316,70 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
         const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
         const bool empty = rb.x > rb.y;
         const float sigma = row_in ? p.sink[(size_t(b) * p.S + i) * p.Hq + h] : 0.f;
-        float m2 = sigma * kLog2e;  // lazily rescaled running maximum, log2 units
+        float m2 = sigma * kLog2e;  // running maximum, log2 units
         float l = 1.f;              // running denominator; the sink contributes exp(0)
+        bool seen = false;          // some earlier step held an unmasked key of this row
 
-        uint8_t* band = smem + L::BAND_OFF + s * BAND_BYTES;
-        const int unit = band_unit(r);
-        const uint32_t band_saddr = smem_u32(band) + uint32_t(unit) * 16u;
-        const uint32_t* band_words = reinterpret_cast<const uint32_t*>(band + unit * 16);
-        const int m_r = (r + 1) & 7;   // misalignment of the row's window start (delta % 8 == 0)
+        uint8_t* band0 = smem + L::BAND_OFF + (2 * s) * BAND_BYTES;
+        const int row_off = band_slot(r) * BAND_PITCH;
+        const int m_r = (r + 1) & 7;   // misalignment of the row's window start
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
         const uint16_t* prof_row =
             (p.R > 0 && row_in && !empty) ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) : nullptr;
-
-        auto band_needed = [&](int n) { return (t_begin + n) * BN + wq * 32 - 127 < p.R; };
+        auto delta_of = [&](int n) { return BN * (u_begin + n) - BN; };
+        // the warp's smallest distance is delta + 32 wq - 63: no profile entry if >= R
+        auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - (BN - 1) < p.R; };
+        // copy this row's window of step n into band buffer (n & 1); always commits a
+        // group so that exactly two groups are outstanding at every wait below
         auto issue_band = [&](int n) {
-            const int x0 = (t_begin + n) * BN + r - 127 - m_r;
+            if (n < n_steps && band_needed(n)) {
+                const uint32_t dst = smem_u32(band0 + (n & 1) * BAND_BYTES + row_off);
+                const int x0 = delta_of(n) + r - (BN - 1) - m_r;
 #pragma unroll
-            for (int q = 0; q < BAND_CHUNKS; ++q) {
-                const int d0 = x0 + 8 * q;
-                const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
-                const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                cp_async_16(band_saddr + 16u * q, src, inb ? 16u : 0u);
+                for (int q = 0; q < BAND_CHUNKS; ++q) {
+                    const int d0 = x0 + 8 * q;
+                    const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
+                    const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
+                    cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                }
             }
             cp_async_commit();
         };
+        // warm the L2 with the window of step n, well before its copy is issued
+        auto prefetch_band = [&](int n) {
+            if (n < n_steps && prof_row != nullptr) {
+                const int x0 = delta_of(n) + r - (BN - 1) - m_r;
+                if (x0 + 8 * BAND_CHUNKS > 0 && x0 < p.R) {
+                    const int lo = max(x0, 0), hi = min(x0 + 8 * BAND_CHUNKS, p.R) - 1;
+                    prefetch_l2(prof_row + lo);                    // the 144-byte window
+                    prefetch_l2(prof_row + min(lo + 64, hi));      // touches at most three
+                    prefetch_l2(prof_row + hi);                    // 128-byte lines
+                }
+            }
+        };
 
-        if (n_steps > 0 && band_needed(0)) issue_band(0);
+        issue_band(0);
+        issue_band(1);
+        prefetch_band(2);
+        prefetch_band(3);
         bool ok = true;
         for (int n = 0; n < n_steps; ++n) {
-            const int j0 = i0g - (t_begin + n) * BN;
-            const bool my_full = empty || (rb.x <= j0 && rb.y >= j0 + BN - 1);
+            const int buf = n & 1;
+            const int jk = key0(n);
+            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + BN - 1);
             const bool need_mask = !__all_sync(0xffffffffu, my_full);
             const bool use_band = band_needed(n);
-            if (!warp_wait(&s_full[s], n & 1, ctl, p.err, kErrFwdS, p.timeout_ns)) {
+            prefetch_band(n + 4);
+            if (!warp_wait(&s_full[2 * s + buf], (n >> 1) & 1, ctl, p.err, kErrFwdS, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             if (wq == 0 && lane == 0) IRA_TRACE(p, 11 + 3 * s, n);
             tc_fence_after();
-            uint32_t x[128];
-            tmem_ld32(tmem + lane_base + L::s_col(s) + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-            tmem_ld32(tmem + lane_base + L::s_col(s) + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-            tmem_ld32(tmem + lane_base + L::s_col(s) + 64, *reinterpret_cast<uint32_t(*)[32]>(&x[64]));
-            tmem_ld32(tmem + lane_base + L::s_col(s) + 96, *reinterpret_cast<uint32_t(*)[32]>(&x[96]));
+            uint32_t x[64];
+            tmem_ld32(tmem + lane_base + L::s_col(s, buf) + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+            tmem_ld32(tmem + lane_base + L::s_col(s, buf) + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
             tmem_wait_ld();
 
             // pass 1: the row maximum, in the units of `coef` (which turns x into log2 units)
@@ -321,7 +389,7 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                 // since scale > 0, max(scale * s) = scale * max(s)
                 float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 128; c += 8) {
+                for (int c = 0; c < 64; c += 8) {
                     a0 = fmax3(a0, __uint_as_float(x[c + 0]), __uint_as_float(x[c + 1]));
                     a1 = fmax3(a1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
                     a2 = fmax3(a2, __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
@@ -331,51 +399,53 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                 coef = p.scale_log2;
             } else {
                 // x becomes the logit scale * s + profile bias (natural units), masked
-                if (use_band) cp_async_wait_all();
-                const int c_lo = rb.x - j0, c_hi = rb.y - j0;  // allowed columns of this row
-                const float2 sc2 = make_float2(p.scale, p.scale);
+                uint32_t w[33];
+                if (use_band) {
+                    cp_async_wait_group<1>();  // this step's window (the next step's may fly)
+                    const uint32_t* words =
+                        reinterpret_cast<const uint32_t*>(band0 + buf * BAND_BYTES + row_off) + g_r;
+#pragma unroll
+                    for (int q = 0; q < 33; ++q) w[q] = words[q];
+                }
+                const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
                 float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t w[17];
+                for (int pp = 0; pp < 32; ++pp) {
+                    const int c = 2 * pp;
+                    float b0 = 0.f, b1 = 0.f;
                     if (use_band) {
-#pragma unroll
-                        for (int q = 0; q < 17; ++q) w[q] = band_words[g_r + 48 - 16 * c4 + q];
+                        const uint32_t v = funnel_r(w[31 - pp], w[32 - pp], fshift);
+                        b0 = bf16hi_to_f32(v);  // column c
+                        b1 = bf16lo_to_f32(v);  // column c+1
                     }
-#pragma unroll
-                    for (int pp = 0; pp < 16; ++pp) {
-                        const int c = 32 * c4 + 2 * pp;
-                        float2 bias = make_float2(0.f, 0.f);
-                        if (use_band) {
-                            const uint32_t v = funnel_r(w[15 - pp], w[16 - pp], fshift);
-                            bias.x = bf16hi_to_f32(v);  // column c
-                            bias.y = bf16lo_to_f32(v);  // column c+1
-                        }
-                        float2 y = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2,
-                                              bias);
-                        if (need_mask) {
-                            y.x = (c >= c_lo && c <= c_hi) ? y.x : -INFINITY;
-                            y.y = (c + 1 >= c_lo && c + 1 <= c_hi) ? y.y : -INFINITY;
-                        }
-                        x[c] = __float_as_uint(y.x);
-                        x[c + 1] = __float_as_uint(y.y);
-                        if (pp & 1)
-                            a1 = fmax3(a1, y.x, y.y);
-                        else
-                            a0 = fmax3(a0, y.x, y.y);
+                    float y0 = fmaf(__uint_as_float(x[c]), p.scale, b0);
+                    float y1 = fmaf(__uint_as_float(x[c + 1]), p.scale, b1);
+                    if (need_mask) {
+                        y0 = (c >= c_lo && c <= c_hi) ? y0 : -INFINITY;
+                        y1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? y1 : -INFINITY;
                     }
+                    x[c] = __float_as_uint(y0);
+                    x[c + 1] = __float_as_uint(y1);
+                    if (pp & 1)
+                        a1 = fmax3(a1, y0, y1);
+                    else
+                        a0 = fmax3(a0, y0, y1);
                 }
                 mx = fmaxf(a0, a1);
                 coef = kLog2e;
-                // this row's band buffer is free again: prefetch the next step's window
-                // (band_needed is non-increasing in n, so only this path can need it)
-                if (n + 1 < n_steps && band_needed(n + 1)) issue_band(n + 1);
             }
-
+            // this step's band buffer is consumed: fetch the window of step n + 2 into it
+            issue_band(n + 2);
             if (wq == 0 && lane == 0) IRA_TRACE(p, 12 + 3 * s, n);
-            // running maximum (log2 units): exact on the first step, lazily moved after
+
+            // running maximum (log2 units): exact on the row's first step with an
+            // unmasked key (so its largest probability is exactly 1 in BF16), lazily
+            // moved after. Until then every P of the row was 0, so its O row is 0 and
+            // needs no rescale.
             const float mx2 = mx * coef;
-            const bool bump = (n == 0) ? (mx2 > m2) : (mx2 > m2 + kRescaleThreshold);
+            const bool first = !seen;
+            seen = seen || (mx2 > -INFINITY);
+            const bool bump = first ? (mx2 > m2) : (mx2 > m2 + kRescaleThreshold);
             float alpha = 1.f;
             if (bump) {
                 alpha = ex2_approx(m2 - mx2);
@@ -384,16 +454,17 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
             }
             const float base = (m2 == -INFINITY) ? 0.f : m2;
 
-            // pass 2: probabilities, row sum, BF16 pack, store P over the S columns
+            // pass 2: probabilities, row sum, BF16 pack, store P over this step's S buffer
             const float2 c2 = make_float2(coef, coef), nb2 = make_float2(-base, -base);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int c = 32 * q + 2 * u;
-                    const float2 t = __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), c2, nb2);
+                    const float2 t =
+                        __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), c2, nb2);
                     const float2 pr = make_float2(ex2_approx(t.x), ex2_approx(t.y));
                     pk[u] = pack_bf16x2(pr.x, pr.y);
                     if (u & 1)
@@ -401,13 +472,20 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
                     else
                         acc0 = __fadd2_rn(acc0, pr);
                 }
-                tmem_st16(tmem + lane_base + L::s_col(s) + 16 * q, pk);
+                tmem_st16(tmem + lane_base + L::s_col(s, buf) + 16 * q, pk);
             }
             l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
 
-            // rescale O when a row of this warp moved its maximum (O of step n-1 is complete:
-            // the S MMA of this step was committed after it)
-            if (n > 0 && __any_sync(0xffffffffu, bump)) {
+            // rescale O when a row of this warp moved its maximum; the PV product of
+            // step n-1 must be complete first (the one of step n waits for this P).
+            // The parity wait is unambiguous: S(n), already waited for, was issued
+            // after PV(n-2), and PV(n) cannot start before this warp's arrival.
+            if (__any_sync(0xffffffffu, bump && !first)) {
+                if (!warp_wait(&o_done[s], (n - 1) & 1, ctl, p.err, kErrFwdO, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
@@ -421,7 +499,7 @@ __global__ void __launch_bounds__(32 * ((NH == 2) ? 12 : 6), 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[s]);
+            if (lane == 0) mbar_arrive(&p_full[2 * s + buf]);
             if (wq == 0 && lane == 0) IRA_TRACE(p, 13 + 3 * s, n);
         }
         cp_async_wait_all();

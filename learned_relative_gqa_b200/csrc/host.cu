@@ -286,9 +286,9 @@ inkling_status inkling_rel_attn_fwd(const inkling_rel_attn_dims* dims, const uin
     CUtensorMap tq, tk, tv;
     if (!encode_bhtd(&tq, q, dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, 128) ||
         !encode_bhtd(&tk, no_keys ? q : k, dims->batch, no_keys ? 1 : dims->seq_k,
-                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 128) ||
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64) ||
         !encode_bhtd(&tv, no_keys ? q : v, dims->batch, no_keys ? 1 : dims->seq_k,
-                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 128))
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64))
         return INKLING_ERR_CUDA;
 
     LaunchTimer tm(st);
