@@ -71,22 +71,78 @@ def ncu_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """SM clock, power and clock-event reasons sampled every few milliseconds during the
+    timed region, through NVML from a background thread (the timed loop spends its time
+    in CUDA synchronisation, which releases the GIL). Falls back to ``nvidia-smi -lms``
+    when NVML is unavailable. Samples are also written to ``path`` as CSV."""
 
-    def __init__(self, index: int, path: str):
-        self.path = path
-        self.proc = None
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
+    def __init__(self, device_index: int, path: str, period_s: float = 0.004):
+        import threading
+        self.path, self.period = path, period_s
+        self.rows, self.proc, self.thread = [], None, None
+        self.stop_evt = threading.Event()
         try:
-            self.f = open(path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.nvml, self.handle = pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.sample()  # one sample before the timed region starts
+            self.rows.clear()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
         except Exception:
-            self.proc = None
+            self.nvml = None
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            try:
+                self.f = open(path, "w")
+                self.proc = subprocess.Popen(["nvidia-smi", f"--id={device_index}", f"--query-gpu={q}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                             stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+
+    def sample(self):
+        nv = self.nvml
+        sm = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+        try:
+            mask = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+        except Exception:
+            mask = int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle))
+        power = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+        self.rows.append((time.time(), sm, self.max_mhz, power, mask))
+
+    def _loop(self):
+        while not self.stop_evt.is_set():
+            try:
+                self.sample()
+            except Exception:
+                return
+            time.sleep(self.period)
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            try:
+                self.sample()  # the state right at the end of the timed region
+            except Exception:
+                pass
+            with open(self.path, "w") as f:
+                f.write("time,sm_mhz,sm_max_mhz,power_w,reasons_mask\n")
+                for r in self.rows:
+                    f.write(f"{r[0]:.4f},{r[1]:.0f},{r[2]:.0f},{r[3]:.1f},{r[4]:#x}\n")
+            if not self.rows:
+                return None
+            sm = sorted(r[1] for r in self.rows)
+            reasons = sorted({name for r in self.rows for bit, name in self.REASONS.items() if r[4] & bit})
+            return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(self.rows), "source": "nvml"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -108,7 +164,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
         return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi"}
 
 
 def cpu_cores() -> int:

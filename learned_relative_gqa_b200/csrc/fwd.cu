@@ -279,13 +279,16 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     issue_s(n);
                     mma_commit(&k_empty[n % KSLOTS]);
                 }
+                auto wait_v = [&](int n) {
+                    return mbar_wait(&v_full[n % VSLOTS], (n / VSLOTS) & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
+                };
+                // The tiles of step n + 1 are awaited right after the MMAs of step n are
+                // queued, so that the path from P(n) to S(n+2) holds one wait only.
+                ok = ok && wait_v(0) && (n_steps <= 2 || wait_k(2));
                 for (int n = 0; ok && n < n_steps; ++n) {
-                    ok = mbar_wait(&v_full[n % VSLOTS], (n / VSLOTS) & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
-                    if (s == 0) IRA_TRACE(p, 10, n);
                     // one barrier per S buffer: the softmax may already have finished
                     // step n + 1 (whose S was issued before this wait)
-                    ok = ok && mbar_wait(&p_full[2 * s + (n & 1)], (n >> 1) & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
-                    if (ok && n + 2 < n_steps) ok = wait_k(n + 2);
+                    ok = mbar_wait(&p_full[2 * s + (n & 1)], (n >> 1) & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
                     if (!ok) break;
                     IRA_TRACE(p, 7 + s, n);
                     tc_fence_after();
@@ -295,6 +298,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                         issue_s(n + 2);
                         mma_commit(&k_empty[(n + 2) % KSLOTS]);
                     }
+                    if (n + 1 < n_steps) ok = wait_v(n + 1) && (n + 3 >= n_steps || wait_k(n + 3));
+                    if (s == 0) IRA_TRACE(p, 10, n + 1);
                 }
                 // O is final once every PV product has completed
                 if (ok) mma_commit(&o_full[s]);
