@@ -18,8 +18,12 @@
 //     has exactly one allowed key.
 //   * dq: one CTA per (batch, query head, 128-row query tile) over 64-key
 //     tiles: S = Q K^T, dP = dO V^T, dQ += dS K (dS from TMEM). No atomics.
-// In both, S/dP are double buffered in TMEM and two softmax warpgroups take
-// alternate steps, so the MMAs of one step overlap the other's elementwise work.
+// In both, S/dP are double buffered in TMEM and the two elementwise warpgroups
+// split the columns of every step (each owns half of them, with its own staged
+// profile rows), so the MMAs of step n+1 run while step n is being processed.
+#include <cstddef>
+#include <type_traits>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -40,18 +44,23 @@ namespace kv {
 
 constexpr int BK = 128;              // keys per CTA (TMEM lanes)
 constexpr int BQ = 64;               // queries per step
-constexpr int BAND_CHUNKS = 17;      // 16-B chunks per band row
-constexpr int BAND_PITCH = BAND_CHUNKS * 16;
-constexpr int BAND_BYTES = BQ * BAND_PITCH;
+constexpr int HALF = BQ / 2;         // query columns per elementwise warpgroup
+constexpr int BAND_LEN = 136;        // bf16 per band row: 128 distances + up to 7 of misalignment
+constexpr int BAND_PITCH = BAND_LEN * 2;
+// Band rows of a step, fetched as 9 TMA boxes of 8 rows (2176 B each, so every box
+// starts on the 128-byte boundary a tensor copy needs): row dm + c holds column c.
+constexpr int BAND_BOXES = BQ / 8 + 1;
+constexpr int BAND_BYTES = BAND_BOXES * 8 * BAND_PITCH;
+constexpr int NB = 3;                // band / column-info buffers
 constexpr int KTILE = BK * 128;      // [128 rows x 64 bf16] box
 constexpr int QTILE = BQ * 128;      // [64 rows x 64 bf16] box
 constexpr int NST = 3;               // Q / dO stages (two steps of lookahead)
 
+// per query column of a step: allowed key range (lo, hi), -lse*log2(e), -Dv
 struct StepInfo {
-    int lo[BQ];
-    int hi[BQ];
-    float lse2[BQ];
-    float dv[BQ];
+    int2 rb[BQ];
+    float nlse2[BQ];
+    float ndv[BQ];
 };
 
 template <int D>
@@ -61,11 +70,12 @@ struct Layout {
     static constexpr int V_OFF = K_OFF + KB * KTILE;
     static constexpr int Q_OFF = V_OFF + KB * KTILE;             // 2 stages
     static constexpr int DO_OFF = Q_OFF + NST * KB * QTILE;      // NST stages
-    static constexpr int BAND_OFF = DO_OFF + NST * KB * QTILE;   // 2 buffers (one per warpgroup)
-    static constexpr int INFO_OFF = BAND_OFF + 2 * BAND_BYTES;   // 2 StepInfo
-    static constexpr int BAR_OFF = INFO_OFF + 2 * int(sizeof(StepInfo));
-    // kv_full, qd_full[NST], qd_empty[NST], s_full[2], p_full[2], acc_full, drain
-    static constexpr int NBARS = 7 + 2 * NST;
+    static constexpr int BAND_OFF = DO_OFF + NST * KB * QTILE;   // NB buffers
+    static constexpr int INFO_OFF = BAND_OFF + NB * BAND_BYTES;  // NB buffers
+    static constexpr int BAR_OFF = INFO_OFF + NB * int(sizeof(StepInfo));
+    // kv_full, qd_full[NST], qd_empty[NST], s_full[2], p_full[2], acc_full, drain,
+    // band_full[NB], band_empty[NB]
+    static constexpr int NBARS = 7 + 2 * NST + 2 * NB;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -80,10 +90,10 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const AttnParams p, const int num_ktiles) {
+                const __grid_constant__ CUtensorMap tm_band, const AttnParams p, const int num_ktiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9, BAND_WARP = 10;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
@@ -96,6 +106,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* p_full = bars + 3 + 2 * NST;     // [2]
     uint64_t* acc_full = bars + 5 + 2 * NST;
     uint64_t* drain = bars + 6 + 2 * NST;
+    uint64_t* band_full = bars + 7 + 2 * NST;       // [NB]
+    uint64_t* band_empty = band_full + NB;          // [NB]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -116,10 +128,14 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(&s_full[u], 1);
-            mbar_init(&p_full[u], 4);
+            mbar_init(&p_full[u], 8);
         }
         mbar_init(acc_full, 1);
         mbar_init(drain, 1);
+        for (int u = 0; u < NB; ++u) {
+            mbar_init(&band_full[u], 1);
+            mbar_init(&band_empty[u], 8);  // every elementwise warp
+        }
         ctl->abort = 0;
         tinfo[0] = 0x7FFFFFFF;  // first query tile that sees the key tile
         tinfo[1] = -1;          // last
@@ -153,11 +169,13 @@ __global__ void __launch_bounds__(384, 1)
     auto step_h = [&](int n) { return g * G + n / n_qt; };
     auto step_qt = [&](int n) { return qt_first + n % n_qt; };
 
-    // Launched with 384 x 168 registers; warpgroup 2 (producer, MMA issuer, two idle
-    // warps) gives its share to the two elementwise warpgroups
-    // (128 x 40 + 256 x 232 = 384 x 168). Each change sits at the top of its branch.
+    // Launched with 384 x 168 registers; warpgroup 2 (tile producer, MMA issuer, band
+    // producer, an idle warp) gives part of its share to the two elementwise warpgroups
+    // (128 x 56 + 256 x 224 = 384 x 168). Each change sits at the top of its branch.
+    // A step whose smallest distance delta - 127 is >= R has no profile entry.
+    auto band_used = [&](int n) { return p.R > 0 && p.q_off + step_qt(n) * BQ - j0 - (BK - 1) < p.R; };
     if (warp >= 8) {
-        setmaxnreg_dec<40>();
+        setmaxnreg_dec<56>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -185,6 +203,58 @@ __global__ void __launch_bounds__(384, 1)
             mbar_wait_drain(kv_full, 0, p.timeout_ns);
             for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
                 mbar_wait_drain(&qd_full[n % NST], (n / NST) & 1, p.timeout_ns);
+        }
+    } else if (warp == BAND_WARP) {
+        // ------------------------------------------------------------ band producer
+        // Per step: the column info (allowed key range, -lse log2 e, -Dv of the 64
+        // query rows) by plain loads, then the band: query column c needs the 136
+        // profile entries from distance delta + c - 127 - m, m = (delta + c - 127) mod 8
+        // (zero outside [0, R)). The columns with the same start (8 consecutive ones)
+        // form one 8-row TMA box. NB buffers run ahead of the elementwise warps.
+        if (n_steps > 0) {
+            int last = -1;
+            for (int n = 0; n < n_steps; ++n) {
+                const int buf = n % NB;
+                if (!warp_wait(&band_empty[buf], ((n / NB) & 1) ^ 1, ctl, p.err, kErrDkdvQFree, p.timeout_ns)) break;
+                const int h = step_h(n), i0 = step_qt(n) * BQ;
+                StepInfo* info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF) + buf;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int c = lane + 32 * k, i = i0 + c;
+                    int2 rb = make_int2(kEmptyLo, kEmptyHi);
+                    float l2 = 0.f, dv = 0.f;
+                    if (i < p.S) {
+                        rb = p.row_bounds[size_t(b) * p.S + i];
+                        const size_t t = (size_t(b) * p.Hq + h) * p.S + i;
+                        l2 = p.lse2t[t];
+                        dv = p.dvt[t];
+                    }
+                    info->rb[c] = rb;
+                    info->nlse2[c] = -l2;
+                    info->ndv[c] = -dv;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    const bool used = band_used(n);
+                    mbar_arrive_expect_tx(&band_full[buf], used ? BAND_BYTES : 0);
+                    if (used) {
+                        const int delta = p.q_off + i0 - j0;
+                        const int dm = (delta - 127) & 7;
+                        const int x0 = delta - 127 - dm;  // multiple of 8
+                        const int row0 = (b * p.Hq + h) * p.S + i0 - dm;
+                        uint8_t* band = smem + L::BAND_OFF + buf * BAND_BYTES;
+                        // box g: shared rows 8g .. 8g+7 = columns 8g - dm .. 8g - dm + 7
+                        for (int g8 = 0; g8 < BAND_BOXES; ++g8)
+                            tma_load_2d(band + g8 * 8 * BAND_PITCH, &tm_band, &band_full[buf], x0 + 8 * g8, row0 + 8 * g8);
+                    }
+                    IRA_TRACE(p, 34, n);
+                }
+                last = n;
+            }
+            // never leave a copy in flight into shared memory of an exiting CTA
+            if (lane == 0)
+                for (int n = (last >= NB ? last - NB + 1 : 0); n <= last; ++n)
+                    mbar_wait_drain(&band_full[n % NB], (n / NB) & 1, p.timeout_ns);
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0 && n_steps > 0) {
@@ -227,17 +297,19 @@ __global__ void __launch_bounds__(384, 1)
                 IRA_TRACE(p, 23, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
+                // P^T / dS^T of query columns [32 w, 32 w + 32) sit, packed, at the
+                // start of warpgroup w's own S / dP columns
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {
+                    const uint32_t a_off = HALF * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bdo = sdesc_sw128(smem_u32(do_smem(st, 0)) + kk * 2048, QTILE, 1024);
-                    mma_ts(tmem + L::DV_COL, tmem + L::s_col(bb) + kk * 8, bdo, IDESC_ACC,
-                           (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + L::DV_COL, tmem + L::s_col(bb) + a_off, bdo, IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {
+                    const uint32_t a_off = HALF * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bq = sdesc_sw128(smem_u32(q_smem(st, 0)) + kk * 2048, QTILE, 1024);
-                    mma_ts(tmem + L::DK_COL, tmem + L::dp_col(bb) + kk * 8, bq, IDESC_ACC,
-                           (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + L::DK_COL, tmem + L::dp_col(bb) + a_off, bq, IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&qd_empty[st]);
                 IRA_TRACE(p, 24, n);
@@ -248,155 +320,132 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
     } else {
-        setmaxnreg_inc<232>();
+        setmaxnreg_inc<224>();
         // ------------------------------------------------------------ elementwise warpgroups
-        const int w = warp >> 2;       // this warpgroup takes steps n with n % 2 == w
+        const int w = warp >> 2;       // this warpgroup takes query columns [32 w, 32 w + 32) of every step
         const int wq = warp & 3;
         const int r = wq * 32 + lane;  // key row (TMEM lane)
         const int j = j0 + r;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
         const int tid = threadIdx.x & 127;
-        uint8_t* band = smem + L::BAND_OFF + w * BAND_BYTES;
-        StepInfo* info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF) + w;
+        const int cw = HALF * w;       // first query column of this warpgroup
 
-        // stage the profile band (query rows of the step, distance window) and row info
-        auto stage = [&](int n) {
-            const int h = step_h(n), i0 = step_qt(n) * BQ;
-            const int delta = p.q_off + i0 - j0;
-            for (int id = tid; id < BQ * BAND_CHUNKS; id += 128) {
-                const int c = id / BAND_CHUNKS, q = id % BAND_CHUNKS;
-                const int i = i0 + c;
-                const int m_c = (delta + c - 127) & 7;
-                const int d0 = delta + c - 127 - m_c + 8 * q;
-                const bool inb = p.R > 0 && i < p.S && d0 >= 0 && d0 < p.R;
-                const void* src = inb ? static_cast<const void*>(p.profiles +
-                                                                 ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) + d0)
-                                      : p.safe_src;
-                cp_async_16(smem_u32(band + c * BAND_PITCH + 16 * q), src, inb ? 16u : 0u);
-            }
-            cp_async_commit();
-            if (tid < BQ) {
-                const int i = i0 + tid;
-                int2 rb = make_int2(kEmptyLo, kEmptyHi);
-                float l2 = 0.f, dv = 0.f;
-                if (i < p.S) {
-                    rb = p.row_bounds[size_t(b) * p.S + i];
-                    const size_t t = (size_t(b) * p.Hq + h) * p.S + i;
-                    l2 = p.lse2t[t];
-                    dv = p.dvt[t];
-                }
-                info->lo[tid] = rb.x;
-                info->hi[tid] = rb.y;
-                info->lse2[tid] = l2;
-                info->dv[tid] = dv;
-            }
-        };
-
-        if (w < n_steps) stage(w);
         bool ok = true;
-        for (int n = w; n < n_steps; n += 2) {
-            const int bb = n & 1;
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 l2e = make_float2(kLog2e, kLog2e);
+        for (int n = 0; n < n_steps; ++n) {
+            const int bb = n & 1, buf = n % NB;
             const int h = step_h(n), qt = step_qt(n), i0 = qt * BQ;
             const int delta = p.q_off + i0 - j0;
             const TileBounds tb = p.tile_bounds[size_t(b) * t64 + qt];
             const bool full = tb.n_nonempty == BQ && tb.max_lo <= j0 && tb.min_hi >= j0 + BK - 1;
-            // all four warps reach this vote whatever their wait returned, so the
-            // warpgroup leaves the loop together (the vote doubles as the barrier
-            // that publishes the staged band and row info)
-            const bool got = warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDkdvS, p.timeout_ns);
-            cp_async_wait_all();
-            if (!named_bar_and(1 + w, 128, got)) {
+            const bool used = band_used(n);
+            // warp-uniform waits: S / dP of the step, then its band rows and column info
+            if (!warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDkdvS, p.timeout_ns) ||
+                !warp_wait(&band_full[buf], (n / NB) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             if (tid == 0) IRA_TRACE(p, 25 + 3 * w, n);
             tc_fence_after();
-            uint32_t sv[64], dp[64];
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+            uint32_t sv[HALF], dp[HALF];
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + cw, sv);
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + cw, dp);
+
+            // Band reads. Column c = cw + cl reads element (m + 127 - r) of shared band row
+            // dm + c, where m = (dm + c) mod 8 repeats every 8 columns (cw is a multiple
+            // of 8): eight per-step shared addresses plus compile-time offsets cover them all.
+            const int dm = (delta - 127) & 7;
+            const uint32_t band_s = smem_u32(smem + L::BAND_OFF + buf * BAND_BYTES + (dm + cw) * BAND_PITCH);
+            uint32_t baddr[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) baddr[u] = band_s + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r);
+            const uint32_t info_s = smem_u32(smem + L::INFO_OFF + buf * int(sizeof(StepInfo)));
+            // dprofiles[b, h, i0 + c, delta + c - r] for column c = cw + cl: the address of
+            // column cl is dbase + cl (R + 1) floats
+            char* const dbase = reinterpret_cast<char*>(
+                p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0 + cw) * size_t(p.R) + (delta + cw - r));
+            const uint32_t dstride4 = 4u * uint32_t(p.R + 1);
+            // d = delta + c - r < R  <=>  c < R - delta + r (no limit when the whole step is inside R)
+            const bool inside = delta + BQ - 1 < p.R;
+            const int cl_lim = (inside ? BQ : p.R - delta + r) - cw;
             tmem_wait_ld();
             if (tid == 0) IRA_TRACE(p, 31, n);
-
-            // Band reads. Column cc reads element (m_cc + 127 - r) of band row cc, where
-            // m_cc = (delta + cc - 127) mod 8 repeats every 8 columns: eight per-step
-            // base pointers (one per cc mod 8) plus compile-time offsets cover them all.
-            const int dm = (delta - 127) & 7;
-            const uint16_t* bptr[8];
+            uint32_t pk[HALF / 2], dk[HALF / 2];
+            // USED: the step reads profile entries; PLAIN: every (key, query) pair of the
+            // step is allowed and inside R, so there is no mask and no store predicate
+            auto math = [&](auto used_c, auto plain_c) {
+                constexpr bool USED = decltype(used_c)::value, PLAIN = decltype(plain_c)::value;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                bptr[u] = reinterpret_cast<const uint16_t*>(band + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r));
-            // dprofiles[b, h, i0 + c, delta + c - r] for column c: one pointer stepped by R + 1
-            float* dptr = p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) + (delta - r);
-            const size_t dstride = size_t(p.R) + 1;
-            // d = delta + c - r < R  <=>  c < R - delta + r  (no limit when the whole step is inside R)
-            const int c_lim = (delta + BQ - 1 < p.R) ? BQ : p.R - delta + r;
-            const float* lse2v = info->lse2;
-            const float* dvv = info->dv;
-            uint32_t pk[32], dk[32];
+                for (int c16 = 0; c16 < HALF / 16; ++c16) {
+                    // loads of this 16-column chunk, issued together
+                    float nl_c[16], nv_c[16], bias_c[16];
+                    int lo_c[16], hi_c[16];
 #pragma unroll
-            for (int c16 = 0; c16 < BQ / 16; ++c16) {
-                // loads of this 16-column chunk, issued together
-                float lse_c[16], dv_c[16], bias_c[16];
-                int lo_c[16], hi_c[16];
-#pragma unroll
-                for (int u4 = 0; u4 < 4; ++u4) {  // 128-bit broadcast reads of four columns
-                    const float4 l4 = reinterpret_cast<const float4*>(lse2v)[4 * c16 + u4];
-                    const float4 v4 = reinterpret_cast<const float4*>(dvv)[4 * c16 + u4];
-                    lse_c[4 * u4 + 0] = l4.x; lse_c[4 * u4 + 1] = l4.y; lse_c[4 * u4 + 2] = l4.z; lse_c[4 * u4 + 3] = l4.w;
-                    dv_c[4 * u4 + 0] = v4.x; dv_c[4 * u4 + 1] = v4.y; dv_c[4 * u4 + 2] = v4.z; dv_c[4 * u4 + 3] = v4.w;
-                    if (!full) {
-                        const int4 a4 = reinterpret_cast<const int4*>(info->lo)[4 * c16 + u4];
-                        const int4 b4 = reinterpret_cast<const int4*>(info->hi)[4 * c16 + u4];
-                        lo_c[4 * u4 + 0] = a4.x; lo_c[4 * u4 + 1] = a4.y; lo_c[4 * u4 + 2] = a4.z; lo_c[4 * u4 + 3] = a4.w;
-                        hi_c[4 * u4 + 0] = b4.x; hi_c[4 * u4 + 1] = b4.y; hi_c[4 * u4 + 2] = b4.z; hi_c[4 * u4 + 3] = b4.w;
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int c = 16 * c16 + u;
-                    bias_c[u] = __uint_as_float(uint32_t(bptr[c & 7][1088 * (c >> 3)]) << 16);
-                }
-#pragma unroll
-                for (int u = 0; u < 16; u += 2) {
-                    const int c = 16 * c16 + u;
-                    float pr[2], ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float t = fmaf(bias_c[u + e], kLog2e, -lse_c[u + e]);
-                        float pv = ex2_approx(fmaf(__uint_as_float(sv[c + e]), p.scale_log2, t));
-                        bool ok = true;
-                        if (!full) {
-                            ok = j >= lo_c[u + e] && j <= hi_c[u + e];
-                            pv = ok ? pv : 0.f;
+                    for (int u4 = 0; u4 < 4; ++u4) {  // 128-bit broadcast reads of four columns
+                        const int c = cw + 16 * c16 + 4 * u4;
+                        const float4 l4 = lds_f32x4(info_s + offsetof(StepInfo, nlse2) + 4 * c);
+                        const float4 v4 = lds_f32x4(info_s + offsetof(StepInfo, ndv) + 4 * c);
+                        nl_c[4 * u4 + 0] = l4.x; nl_c[4 * u4 + 1] = l4.y; nl_c[4 * u4 + 2] = l4.z; nl_c[4 * u4 + 3] = l4.w;
+                        nv_c[4 * u4 + 0] = v4.x; nv_c[4 * u4 + 1] = v4.y; nv_c[4 * u4 + 2] = v4.z; nv_c[4 * u4 + 3] = v4.w;
+                        if (!PLAIN) {
+                            const int4 a4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c);
+                            const int4 b4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c + 16);
+                            lo_c[4 * u4 + 0] = a4.x; hi_c[4 * u4 + 0] = a4.y; lo_c[4 * u4 + 1] = a4.z; hi_c[4 * u4 + 1] = a4.w;
+                            lo_c[4 * u4 + 2] = b4.x; hi_c[4 * u4 + 2] = b4.y; lo_c[4 * u4 + 3] = b4.z; hi_c[4 * u4 + 3] = b4.w;
                         }
-                        const float dsv = pv * (__uint_as_float(dp[c + e]) - dv_c[u + e]);
-                        if (ok && c + e < c_lim) __stcs(dptr, dsv);
-                        dptr += dstride;
-                        pr[e] = pv;
-                        ds[e] = dsv;
                     }
-                    pk[c >> 1] = pack_bf16x2(pr[0], pr[1]);
-                    dk[c >> 1] = pack_bf16x2(ds[0], ds[1]);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int cl = 16 * c16 + u;
+                        bias_c[u] = USED ? __uint_as_float(lds_u16(baddr[cl & 7] + BAND_PITCH * 8 * (cl >> 3)) << 16) : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; u += 2) {
+                        const int cl = 16 * c16 + u;
+                        // log2-domain logit, probability, dS = P (dP - Dv), two columns at a time
+                        float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[cl]), __uint_as_float(sv[cl + 1])), sl2,
+                                              make_float2(nl_c[u], nl_c[u + 1]));
+                        if (USED) z = __ffma2_rn(make_float2(bias_c[u], bias_c[u + 1]), l2e, z);
+                        float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+                        bool ok0 = true, ok1 = true;
+                        if (!PLAIN) {
+                            ok0 = uint32_t(j - lo_c[u]) <= uint32_t(hi_c[u] - lo_c[u]) && cl < cl_lim;
+                            ok1 = uint32_t(j - lo_c[u + 1]) <= uint32_t(hi_c[u + 1] - lo_c[u + 1]) && cl + 1 < cl_lim;
+                            pr.x = (uint32_t(j - lo_c[u]) <= uint32_t(hi_c[u] - lo_c[u])) ? pr.x : 0.f;
+                            pr.y = (uint32_t(j - lo_c[u + 1]) <= uint32_t(hi_c[u + 1] - lo_c[u + 1])) ? pr.y : 0.f;
+                        }
+                        const float2 ds = __fmul2_rn(
+                            pr, __fadd2_rn(make_float2(__uint_as_float(dp[cl]), __uint_as_float(dp[cl + 1])),
+                                           make_float2(nv_c[u], nv_c[u + 1])));
+                        float* const a0 = reinterpret_cast<float*>(dbase + size_t(uint32_t(cl) * dstride4));
+                        float* const a1 = reinterpret_cast<float*>(dbase + size_t(uint32_t(cl + 1) * dstride4));
+                        if (PLAIN || ok0) __stcs(a0, ds.x);
+                        if (PLAIN || ok1) __stcs(a1, ds.y);
+                        pk[cl >> 1] = pack_bf16x2(pr.x, pr.y);
+                        dk[cl >> 1] = pack_bf16x2(ds.x, ds.y);
+                    }
                 }
+            };
+            using T_ = std::true_type;
+            using F_ = std::false_type;
+            if (used) {
+                if (full && inside) math(T_{}, T_{}); else math(T_{}, F_{});
+            } else {
+                if (full && inside) math(F_{}, T_{}); else math(F_{}, F_{});
             }
             if (tid == 0) IRA_TRACE(p, 32, n);
-            tmem_st16(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-            tmem_st16(tmem + lane_base + L::s_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
+            tmem_st16(tmem + lane_base + L::s_col(bb) + cw, pk);
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + cw, dk);
             tmem_wait_st();
-            if (tid == 0) IRA_TRACE(p, 33, n);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[bb]);
+            if (lane == 0) {
+                mbar_arrive(&p_full[bb]);
+                mbar_arrive(&band_empty[buf]);
+            }
             if (tid == 0) IRA_TRACE(p, 26 + 3 * w, n);
-            named_bar_sync(1 + w, 128);  // band and info of this step fully consumed
-            if (n + 2 < n_steps) stage(n + 2);
-            if (tid == 0) IRA_TRACE(p, 27 + 3 * w, n);
         }
-        cp_async_wait_all();
 
         // ---- epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV ----
         if (ok && n_steps > 0) {
@@ -440,7 +489,7 @@ __global__ void __launch_bounds__(384, 1)
 
 template <int D>
 cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                   const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
+                   const CUtensorMap& tm_do, const CUtensorMap& tm_band, const AttnParams& p, cudaStream_t st) {
     using L = Layout<D>;
     auto kern = dkdv_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
@@ -448,7 +497,7 @@ cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUten
     const int nkt = (p.Skv + BK - 1) / BK;
     const long long grid = (long long)nkt * p.B * p.Hkv;
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nkt);
+    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, tm_band, p, nkt);
     return cudaGetLastError();
 }
 
@@ -461,7 +510,8 @@ namespace dqk {
 
 constexpr int BM = 128;               // query rows per CTA (TMEM lanes)
 constexpr int BN = 64;                // keys per step
-constexpr int BAND_CHUNKS = 9;        // 72 bf16 per row window
+constexpr int HALF = BN / 2;          // key columns per elementwise warpgroup
+constexpr int BAND_CHUNKS = 5;        // 40 bf16 per row window (32 columns + misalignment)
 constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
 constexpr int BAND_BYTES = BAND_UNITS * 16;
 constexpr int QTILE = BM * 128;       // [128 x 64 bf16]
@@ -477,8 +527,8 @@ struct Layout {
     static constexpr int DO_OFF = Q_OFF + KB * QTILE;
     static constexpr int K_OFF = DO_OFF + KB * QTILE;          // NST stages
     static constexpr int V_OFF = K_OFF + NST * KB * KTILE;     // NST stages
-    static constexpr int BAND_OFF = V_OFF + NST * KB * KTILE;  // 2 buffers (one per warpgroup)
-    static constexpr int BAR_OFF = BAND_OFF + 2 * BAND_BYTES;
+    static constexpr int BAND_OFF = V_OFF + NST * KB * KTILE;  // [warpgroup][step parity]
+    static constexpr int BAR_OFF = BAND_OFF + 4 * BAND_BYTES;
     // q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], acc_full, drain
     static constexpr int NBARS = 7 + 2 * NST;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
@@ -532,7 +582,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(&s_full[u], 1);
-            mbar_init(&p_full[u], 4);
+            mbar_init(&p_full[u], 8);
         }
         mbar_init(acc_full, 1);
         mbar_init(drain, 1);
@@ -574,9 +624,9 @@ __global__ void __launch_bounds__(384, 1)
 
     // Launched with 384 x 168 registers; warpgroup 2 (producer, MMA issuer, two idle
     // warps) gives its share to the two elementwise warpgroups
-    // (128 x 40 + 256 x 232 = 384 x 168). Each change sits at the top of its branch.
+    // (128 x 80 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
     if (warp >= 8) {
-        setmaxnreg_dec<40>();
+        setmaxnreg_dec<80>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -649,7 +699,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, 0)) + kk * 2048, KTILE, 1024);
-                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + kk * 8, bk, IDESC_DQ,
+                    // dS of key columns [32 w, 32 w + 32) sits, packed, at the start of
+                    // warpgroup w's own dP columns
+                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + HALF * (kk >> 1) + 8 * (kk & 1), bk, IDESC_DQ,
                            (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&kv_empty[st]);
@@ -661,11 +713,12 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
     } else {
-        setmaxnreg_inc<232>();
-        const int w = warp >> 2;
+        setmaxnreg_inc<208>();
+        const int w = warp >> 2;       // this warpgroup takes key columns [32 w, 32 w + 32) of every step
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
+        const int cw = HALF * w;
         const int i = i0 + r;
         const bool row_in = i < p.S;
         const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
@@ -674,35 +727,49 @@ __global__ void __launch_bounds__(384, 1)
         const float lse2 = row_in ? p.lse2t[trow] : 0.f;
         const float dvr = row_in ? p.dvt[trow] : 0.f;
 
-        uint8_t* band = smem + L::BAND_OFF + w * BAND_BYTES;
+        // This thread's profile window for its columns, double buffered by step parity:
+        // column c = cw + cl of step n has distance delta(n) + r - c; the 32 columns'
+        // window starts (r + 1) mod 8 elements past a 16-byte boundary.
         const int unit = band_unit(r);
-        const uint32_t band_saddr = smem_u32(band) + uint32_t(unit) * 16u;
-        const uint32_t* band_words = reinterpret_cast<const uint32_t*>(band + unit * 16);
+        auto band_saddr = [&](int buf) {
+            return smem_u32(smem + L::BAND_OFF + (2 * w + buf) * BAND_BYTES) + uint32_t(unit) * 16u;
+        };
         const int m_r = (r + 1) & 7;
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
         const uint16_t* prof_row =
             (p.R > 0 && row_in && !empty) ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) : nullptr;
         // step n has distance offset delta = i0g - key0(n) = 64 (t_begin + n) - 64
-        auto band_needed = [&](int n) { return BN * (t_begin + n) - BN + wq * 32 - (BN - 1) < p.R; };
+        auto delta_of = [&](int n) { return BN * (t_begin + n) - BN; };
+        // the warp's smallest distance in this warpgroup's columns is delta + 32 wq - cw - 31
+        auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - cw - (HALF - 1) < p.R; };
+        // one cp.async group per call, also when nothing is copied
         auto issue_band = [&](int n) {
-            const int x0 = BN * (t_begin + n) - BN + r - (BN - 1) - m_r;
+            if (n < n_steps && band_needed(n)) {
+                const int x0 = delta_of(n) + r - cw - (HALF - 1) - m_r;
+                const uint32_t dst = band_saddr(n & 1);
 #pragma unroll
-            for (int q = 0; q < BAND_CHUNKS; ++q) {
-                const int d0 = x0 + 8 * q;
-                const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
-                const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                cp_async_16(band_saddr + 16u * q, src, inb ? 16u : 0u);
+                for (int q = 0; q < BAND_CHUNKS; ++q) {
+                    const int d0 = x0 + 8 * q;
+                    const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
+                    const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
+                    cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                }
             }
             cp_async_commit();
         };
 
-        if (w < n_steps && band_needed(w)) issue_band(w);
+        issue_band(0);
+        issue_band(1);
         bool ok = true;
-        for (int n = w; n < n_steps; n += 2) {
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 l2e = make_float2(kLog2e, kLog2e);
+        const float2 nl2 = make_float2(-lse2, -lse2);
+        const float2 nv2 = make_float2(-dvr, -dvr);
+        for (int n = 0; n < n_steps; ++n) {
             const int bb = n & 1;
-            const int jk = key0(n);
-            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + BN - 1);
+            const int jk = key0(n) + cw;  // key of this warpgroup's first column
+            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + HALF - 1);
             const bool need_mask = !__all_sync(0xffffffffu, my_full);
             const bool use_band = band_needed(n);
             if (!warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDqS, p.timeout_ns)) {
@@ -711,32 +778,28 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (wq == 0 && lane == 0) IRA_TRACE(p, 45 + 2 * w, n);
             tc_fence_after();
-            uint32_t sv[64], dp[64];
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-            tmem_wait_ld();
-            uint32_t wv[33];
+            uint32_t sv[HALF], dp[HALF];
+            tmem_ld32(tmem + lane_base + L::s_col(bb) + cw, sv);
+            tmem_ld32(tmem + lane_base + L::dp_col(bb) + cw, dp);
+            uint32_t wv[17];
             if (use_band) {
-                cp_async_wait_all();
+                cp_async_wait_group<1>();  // this step's window (the next step's may fly)
+                const uint32_t* words =
+                    reinterpret_cast<const uint32_t*>(smem + L::BAND_OFF + (2 * w + bb) * BAND_BYTES + unit * 16) + g_r;
 #pragma unroll
-                for (int q = 0; q < 33; ++q) wv[q] = band_words[g_r + q];
+                for (int q = 0; q < 17; ++q) wv[q] = words[q];
             }
-            // the row's band buffer is free: prefetch the window of this warpgroup's next step
-            if (n + 2 < n_steps && band_needed(n + 2)) issue_band(n + 2);
-            const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-            const float2 l2e = make_float2(kLog2e, kLog2e);
-            const float2 nl2 = make_float2(-lse2, -lse2);
-            const float2 nv2 = make_float2(-dvr, -dvr);
+            // this step's window is in registers: fetch the one of step n + 2 into its buffer
+            issue_band(n + 2);
+            tmem_wait_ld();
             const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
-            uint32_t dk[32];
+            uint32_t dk[HALF / 2];
 #pragma unroll
-            for (int pp = 0; pp < 32; ++pp) {
+            for (int pp = 0; pp < HALF / 2; ++pp) {
                 const int c = 2 * pp;
                 float2 t = nl2;
                 if (use_band) {
-                    const uint32_t v = funnel_r(wv[31 - pp], wv[32 - pp], fshift);
+                    const uint32_t v = funnel_r(wv[15 - pp], wv[16 - pp], fshift);
                     t = __ffma2_rn(make_float2(bf16hi_to_f32(v), bf16lo_to_f32(v)), l2e, nl2);
                 }
                 const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
@@ -749,8 +812,7 @@ __global__ void __launch_bounds__(384, 1)
                     __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv2));
                 dk[pp] = pack_bf16x2(ds.x, ds.y);
             }
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + 0, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
+            tmem_st16(tmem + lane_base + L::dp_col(bb) + cw, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -819,9 +881,10 @@ cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUten
 }  // namespace bwdk
 
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                            const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
-    return p.D == 128 ? bwdk::kv::launch<128>(tm_q, tm_k, tm_v, tm_do, p, st)
-                      : bwdk::kv::launch<64>(tm_q, tm_k, tm_v, tm_do, p, st);
+                            const CUtensorMap& tm_do, const CUtensorMap& tm_band, const AttnParams& p,
+                            cudaStream_t st) {
+    return p.D == 128 ? bwdk::kv::launch<128>(tm_q, tm_k, tm_v, tm_do, tm_band, p, st)
+                      : bwdk::kv::launch<64>(tm_q, tm_k, tm_v, tm_do, tm_band, p, st);
 }
 
 cudaError_t launch_bwd_dq(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,

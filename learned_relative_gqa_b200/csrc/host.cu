@@ -54,6 +54,21 @@ bool encode_bhtd(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Profiles [B, Hq, S, R] as R-long rows, in boxes of 8 rows x 136 entries (the band
+// rows of 8 consecutive query columns: 128 distances plus up to 7 of misalignment);
+// entries outside [0, R) and rows outside the tensor read 0.
+bool encode_band(CUtensorMap* m, const void* base, int64_t rows, int64_t R) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cuuint64_t(R), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(R * 2)};
+    cuuint32_t box[2] = {136u, 8u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Last CUDA error seen by an entry point of this thread (inkling_rel_attn_last_cuda_error).
@@ -348,6 +363,9 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
         !encode_bhtd(&tk128, kb, B, Skv_m, Hkv_m, D, 128) || !encode_bhtd(&tv128, vb, B, Skv_m, Hkv_m, D, 128) ||
         !encode_bhtd(&tk64, kb, B, Skv_m, Hkv_m, D, 64) || !encode_bhtd(&tv64, vb, B, Skv_m, Hkv_m, D, 64))
         return INKLING_ERR_CUDA;
+    CUtensorMap tband;
+    std::memset(&tband, 0, sizeof(tband));
+    if (dims->rel_extent > 0 && !encode_band(&tband, profiles, B * Hq * S, dims->rel_extent)) return INKLING_ERR_CUDA;
 
     LaunchTimer tm(st);
     s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
@@ -371,7 +389,7 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     p.dk = dk;
     p.dv = dv;
     p.dprofiles = dprofiles;
-    e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, p, st) : cudaSuccess; });
+    e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, tband, p, st) : cudaSuccess; });
     if (e != cudaSuccess) return INKLING_ERR_CUDA;
     return cuda_status(tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st); }));
 }

@@ -26,9 +26,11 @@ cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st)
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const AttnParams& p, cudaStream_t st);
 
-// Backward attention. dkdv: tm_k / tm_v box {64,1,128,1}, tm_q / tm_do box {64,1,64,1}.
+// Backward attention. dkdv: tm_k / tm_v box {64,1,128,1}, tm_q / tm_do box {64,1,64,1},
+// tm_band: profiles as {R, B*Hq*S} with box {136, 8} (unused when R == 0).
 cudaError_t launch_bwd_dkdv(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                            const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st);
+                            const CUtensorMap& tm_do, const CUtensorMap& tm_band, const AttnParams& p,
+                            cudaStream_t st);
 // dq: tm_q / tm_do box {64,1,128,1}, tm_k / tm_v box {64,1,64,1}.
 cudaError_t launch_bwd_dq(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st);
