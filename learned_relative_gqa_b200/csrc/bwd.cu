@@ -212,6 +212,26 @@ __global__ void __launch_bounds__(384, 1)
         // (zero outside [0, R)). The columns with the same start (8 consecutive ones)
         // form one 8-row TMA box. NB buffers run ahead of the elementwise warps.
         if (n_steps > 0) {
+            // column info of step n in registers (lane handles columns lane and lane + 32),
+            // loaded one step before it is stored so the load latency overlaps the wait
+            int2 rb_r[2];
+            float l2_r[2], dv_r[2];
+            auto load_info = [&](int n) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    rb_r[k] = make_int2(kEmptyLo, kEmptyHi);
+                    l2_r[k] = 0.f;
+                    dv_r[k] = 0.f;
+                    const int i = step_qt(n) * BQ + lane + 32 * k;
+                    if (n < n_steps && i < p.S) {
+                        rb_r[k] = p.row_bounds[size_t(b) * p.S + i];
+                        const size_t t = (size_t(b) * p.Hq + step_h(n)) * p.S + i;
+                        l2_r[k] = p.lse2t[t];
+                        dv_r[k] = p.dvt[t];
+                    }
+                }
+            };
+            load_info(0);
             int last = -1;
             for (int n = 0; n < n_steps; ++n) {
                 const int buf = n % NB;
@@ -220,19 +240,12 @@ __global__ void __launch_bounds__(384, 1)
                 StepInfo* info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF) + buf;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
-                    const int c = lane + 32 * k, i = i0 + c;
-                    int2 rb = make_int2(kEmptyLo, kEmptyHi);
-                    float l2 = 0.f, dv = 0.f;
-                    if (i < p.S) {
-                        rb = p.row_bounds[size_t(b) * p.S + i];
-                        const size_t t = (size_t(b) * p.Hq + h) * p.S + i;
-                        l2 = p.lse2t[t];
-                        dv = p.dvt[t];
-                    }
-                    info->rb[c] = rb;
-                    info->nlse2[c] = -l2;
-                    info->ndv[c] = -dv;
+                    const int c = lane + 32 * k;
+                    info->rb[c] = rb_r[k];
+                    info->nlse2[c] = -l2_r[k];
+                    info->ndv[c] = -dv_r[k];
                 }
+                load_info(n + 1);
                 __syncwarp();
                 if (lane == 0) {
                     const bool used = band_used(n);
@@ -289,6 +302,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (n + 1 < n_steps) {
                     ok = mbar_wait(&qd_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns);
                     if (!ok) break;
+                    IRA_TRACE(p, 35, n + 1);
                     tc_fence_after();
                     issue_sdp(n + 1);
                 }
@@ -688,6 +702,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (n + 1 < n_steps) {
                     ok = mbar_wait(&kv_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
                     if (!ok) break;
+                    IRA_TRACE(p, 49, n + 1);
                     tc_fence_after();
                     issue_sdp(n + 1);
                 }
