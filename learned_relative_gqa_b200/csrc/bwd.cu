@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(384, 1)
                 const __grid_constant__ CUtensorMap tm_band, const AttnParams p, const int num_ktiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9, BAND_WARP = 10;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9, BAND_WARP = 10, MMA_WARP_B = 11;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
@@ -122,16 +122,17 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
+        // stage, score and accumulator barriers complete once both MMA issuers committed
         for (int u = 0; u < NST; ++u) {
             mbar_init(&qd_full[u], 1);
-            mbar_init(&qd_empty[u], 1);
+            mbar_init(&qd_empty[u], 2);
         }
         for (int u = 0; u < 2; ++u) {
-            mbar_init(&s_full[u], 1);
+            mbar_init(&s_full[u], 2);
             mbar_init(&p_full[u], 8);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(drain, 1);
+        mbar_init(acc_full, 2);
+        mbar_init(drain, 2);
         for (int u = 0; u < NB; ++u) {
             mbar_init(&band_full[u], 1);
             mbar_init(&band_empty[u], 8);  // every elementwise warp
@@ -169,13 +170,13 @@ __global__ void __launch_bounds__(384, 1)
     auto step_h = [&](int n) { return g * G + n / n_qt; };
     auto step_qt = [&](int n) { return qt_first + n % n_qt; };
 
-    // Launched with 384 x 168 registers; warpgroup 2 (tile producer, MMA issuer, band
-    // producer, an idle warp) gives part of its share to the two elementwise warpgroups
-    // (128 x 56 + 256 x 224 = 384 x 168). Each change sits at the top of its branch.
+    // Launched with 384 x 168 registers; warpgroup 2 (tile producer, two MMA issuers,
+    // band producer) gives part of its share to the two elementwise warpgroups
+    // (128 x 72 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
     // A step whose smallest distance delta - 127 is >= R has no profile entry.
     auto band_used = [&](int n) { return p.R > 0 && p.q_off + step_qt(n) * BQ - j0 - (BK - 1) < p.R; };
     if (warp >= 8) {
-        setmaxnreg_dec<56>();
+        setmaxnreg_dec<72>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -269,25 +270,30 @@ __global__ void __launch_bounds__(384, 1)
                 for (int n = (last >= NB ? last - NB + 1 : 0); n <= last; ++n)
                     mbar_wait_drain(&band_full[n % NB], (n / NB) & 1, p.timeout_ns);
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == MMA_WARP || warp == MMA_WARP_B) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two issuing threads, one per chain, so that one's waits never starve the
+        // tensor core: A issues S^T = K Q^T and dV += P^T dO, B issues dP^T = V dO^T and
+        // dK += dS^T Q. Each chain overwrites its TMEM buffer only after its own product
+        // that read it (the tensor core runs one thread's MMAs in issue order).
+        const bool is_b = warp == MMA_WARP_B;
         if (lane == 0 && n_steps > 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BQ, 0, 0);
             constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
-            auto issue_sdp = [&](int n) {
+            const uint32_t a_base = smem_u32(is_b ? v_smem(0) : k_smem(0));
+            const uint32_t prod_col = is_b ? L::DK_COL : L::DV_COL;
+            auto col_of = [&](int bb) { return is_b ? L::dp_col(bb) : L::s_col(bb); };
+            auto b_base = [&](int st) { return smem_u32(is_b ? do_smem(st, 0) : q_smem(st, 0)); };
+            auto c_base = [&](int st) { return smem_u32(is_b ? q_smem(st, 0) : do_smem(st, 0)); };
+            auto issue_score = [&](int n) {  // S^T (A) or dP^T (B) of step n
                 const int st = n % NST, bb = n & 1;
+                const uint32_t bs = b_base(st);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const int kb = kk >> 2, kin = kk & 3;
-                    const uint64_t ak = sdesc_sw128(smem_u32(k_smem(kb)) + kin * 32, 16, 1024);
-                    const uint64_t bq = sdesc_sw128(smem_u32(q_smem(st, kb)) + kin * 32, 16, 1024);
-                    mma_ss(tmem + L::s_col(bb), ak, bq, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int kb = kk >> 2, kin = kk & 3;
-                    const uint64_t av = sdesc_sw128(smem_u32(v_smem(kb)) + kin * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(smem_u32(do_smem(st, kb)) + kin * 32, 16, 1024);
-                    mma_ss(tmem + L::dp_col(bb), av, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (kk >> 2) * KTILE + (kk & 3) * 32;
+                    const uint32_t boff = (kk >> 2) * QTILE + (kk & 3) * 32;
+                    mma_ss(tmem + col_of(bb), sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(bs + boff, 16, 1024),
+                           IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[bb]);
                 IRA_TRACE(p, 22, n);
@@ -296,37 +302,32 @@ __global__ void __launch_bounds__(384, 1)
                       mbar_wait(&qd_full[0], 0, ctl, p.err, kErrDkdvQ, p.timeout_ns);
             if (ok) {
                 tc_fence_after();
-                issue_sdp(0);
+                issue_score(0);
             }
             for (int n = 0; ok && n < n_steps; ++n) {
                 if (n + 1 < n_steps) {
                     ok = mbar_wait(&qd_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDkdvQ, p.timeout_ns);
                     if (!ok) break;
-                    IRA_TRACE(p, 35, n + 1);
+                    if (!is_b) IRA_TRACE(p, 35, n + 1);
                     tc_fence_after();
-                    issue_sdp(n + 1);
+                    issue_score(n + 1);
                 }
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDkdvP, p.timeout_ns);
                 if (!ok) break;
-                IRA_TRACE(p, 23, n);
+                if (!is_b) IRA_TRACE(p, 23, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
                 // P^T / dS^T of query columns [32 w, 32 w + 32) sit, packed, at the
                 // start of warpgroup w's own S / dP columns
+                const uint32_t cs = c_base(st);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {
                     const uint32_t a_off = HALF * (kk >> 1) + 8 * (kk & 1);
-                    const uint64_t bdo = sdesc_sw128(smem_u32(do_smem(st, 0)) + kk * 2048, QTILE, 1024);
-                    mma_ts(tmem + L::DV_COL, tmem + L::s_col(bb) + a_off, bdo, IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk) {
-                    const uint32_t a_off = HALF * (kk >> 1) + 8 * (kk & 1);
-                    const uint64_t bq = sdesc_sw128(smem_u32(q_smem(st, 0)) + kk * 2048, QTILE, 1024);
-                    mma_ts(tmem + L::DK_COL, tmem + L::dp_col(bb) + a_off, bq, IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + prod_col, tmem + col_of(bb) + a_off, sdesc_sw128(cs + kk * 2048, QTILE, 1024),
+                           IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&qd_empty[st]);
-                IRA_TRACE(p, 24, n);
+                if (!is_b) IRA_TRACE(p, 24, n);
             }
             if (ok) mma_commit(acc_full);
             mma_commit(drain);
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
     } else {
-        setmaxnreg_inc<224>();
+        setmaxnreg_inc<208>();
         // ------------------------------------------------------------ elementwise warpgroups
         const int w = warp >> 2;       // this warpgroup takes query columns [32 w, 32 w + 32) of every step
         const int wq = warp & 3;
@@ -561,7 +562,7 @@ __global__ void __launch_bounds__(384, 1)
               const AttnParams p, const int num_qtiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9, MMA_WARP_B = 11;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
@@ -590,16 +591,17 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        // a K / V stage is free, and S / dP of a step ready, once both MMA issuers committed
         for (int u = 0; u < NST; ++u) {
             mbar_init(&kv_full[u], 1);
-            mbar_init(&kv_empty[u], 1);
+            mbar_init(&kv_empty[u], 2);
         }
         for (int u = 0; u < 2; ++u) {
-            mbar_init(&s_full[u], 1);
+            mbar_init(&s_full[u], 2);
             mbar_init(&p_full[u], 8);
         }
         mbar_init(acc_full, 1);
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
         ctl->abort = 0;
         const TileBounds* tb = p.tile_bounds + size_t(b) * t64 + 2 * qt;
         int min_lo = tb[0].min_lo, max_hi = tb[0].max_hi, ne = tb[0].n_nonempty;
@@ -636,8 +638,8 @@ __global__ void __launch_bounds__(384, 1)
     auto v_smem = [&](int st, int kb) { return smem + L::V_OFF + (st * KB + kb) * KTILE; };
     auto key0 = [&](int n) { return i0g + BN - (t_begin + n) * BN; };
 
-    // Launched with 384 x 168 registers; warpgroup 2 (producer, MMA issuer, two idle
-    // warps) gives its share to the two elementwise warpgroups
+    // Launched with 384 x 168 registers; warpgroup 2 (producer, two MMA issuers, an idle
+    // warp) gives part of its share to the two elementwise warpgroups
     // (128 x 80 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
     if (warp >= 8) {
         setmaxnreg_dec<80>();
@@ -669,60 +671,66 @@ __global__ void __launch_bounds__(384, 1)
             for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
                 mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.timeout_ns);
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == MMA_WARP || warp == MMA_WARP_B) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two issuing threads so that one's waits never starve the tensor core:
+        // A issues S = Q K^T; B issues dP = dO V^T and dQ += dS K (dS from TMEM). Each
+        // overwrites its S / dP buffer only after the elementwise warps are done with the
+        // step that used it, and B's dQ of that step precedes it in B's issue order.
+        const bool is_b = warp == MMA_WARP_B;
         if (lane == 0 && n_steps > 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
             constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);
-            auto issue_sdp = [&](int n) {
+            const uint32_t a_base = smem_u32(is_b ? do_smem(0) : q_smem(0));
+            auto b_base = [&](int st) { return smem_u32(is_b ? v_smem(st, 0) : k_smem(st, 0)); };
+            auto issue_score = [&](int n) {  // S (A) or dP (B) of step n
                 const int st = n % NST, bb = n & 1;
+                const uint32_t bs = b_base(st);
+                const uint32_t col = is_b ? L::dp_col(bb) : L::s_col(bb);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const int kb = kk >> 2, kin = kk & 3;
-                    const uint64_t aq = sdesc_sw128(smem_u32(q_smem(kb)) + kin * 32, 16, 1024);
-                    const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, kb)) + kin * 32, 16, 1024);
-                    mma_ss(tmem + L::s_col(bb), aq, bk, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int kb = kk >> 2, kin = kk & 3;
-                    const uint64_t ad = sdesc_sw128(smem_u32(do_smem(kb)) + kin * 32, 16, 1024);
-                    const uint64_t bv = sdesc_sw128(smem_u32(v_smem(st, kb)) + kin * 32, 16, 1024);
-                    mma_ss(tmem + L::dp_col(bb), ad, bv, IDESC_S, kk > 0 ? 1u : 0u);
+                    const uint32_t aoff = (kk >> 2) * QTILE + (kk & 3) * 32;
+                    const uint32_t boff = (kk >> 2) * KTILE + (kk & 3) * 32;
+                    mma_ss(tmem + col, sdesc_sw128(a_base + aoff, 16, 1024), sdesc_sw128(bs + boff, 16, 1024), IDESC_S,
+                           kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[bb]);
-                IRA_TRACE(p, 42, n);
+                // A's last read of this K stage
+                if (!is_b) mma_commit(&kv_empty[st]);
+                if (!is_b) IRA_TRACE(p, 42, n);
             };
             bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns) &&
                       mbar_wait(&kv_full[0], 0, ctl, p.err, kErrDqKV, p.timeout_ns);
             if (ok) {
                 tc_fence_after();
-                issue_sdp(0);
+                issue_score(0);
             }
             for (int n = 0; ok && n < n_steps; ++n) {
                 if (n + 1 < n_steps) {
                     ok = mbar_wait(&kv_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
                     if (!ok) break;
-                    IRA_TRACE(p, 49, n + 1);
+                    if (!is_b) IRA_TRACE(p, 49, n + 1);
                     tc_fence_after();
-                    issue_sdp(n + 1);
+                    issue_score(n + 1);
                 }
                 ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
                 if (!ok) break;
+                if (!is_b) continue;
                 IRA_TRACE(p, 43, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
+                const uint32_t ks = smem_u32(k_smem(st, 0));
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bk = sdesc_sw128(smem_u32(k_smem(st, 0)) + kk * 2048, KTILE, 1024);
                     // dS of key columns [32 w, 32 w + 32) sits, packed, at the start of
                     // warpgroup w's own dP columns
-                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + HALF * (kk >> 1) + 8 * (kk & 1), bk, IDESC_DQ,
-                           (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + HALF * (kk >> 1) + 8 * (kk & 1),
+                           sdesc_sw128(ks + kk * 2048, KTILE, 1024), IDESC_DQ, (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&kv_empty[st]);
                 IRA_TRACE(p, 44, n);
             }
-            if (ok) mma_commit(acc_full);
+            if (ok && is_b) mma_commit(acc_full);
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
         }
