@@ -61,6 +61,8 @@ struct StepInfo {
     int2 rb[BQ];
     float nlse2[BQ];
     float ndv[BQ];
+    int full;       // every (key, query) pair of the step is allowed
+    int pad[3];
 };
 
 template <int D>
@@ -217,7 +219,12 @@ __global__ void __launch_bounds__(384, 1)
             // loaded one step before it is stored so the load latency overlaps the wait
             int2 rb_r[2];
             float l2_r[2], dv_r[2];
+            bool full_r = false;
             auto load_info = [&](int n) {
+                if (n < n_steps) {
+                    const TileBounds tb = p.tile_bounds[size_t(b) * t64 + step_qt(n)];
+                    full_r = tb.n_nonempty == BQ && tb.max_lo <= j0 && tb.min_hi >= j0 + BK - 1;
+                }
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     rb_r[k] = make_int2(kEmptyLo, kEmptyHi);
@@ -246,6 +253,7 @@ __global__ void __launch_bounds__(384, 1)
                     info->nlse2[c] = -l2_r[k];
                     info->ndv[c] = -dv_r[k];
                 }
+                if (lane == 0) info->full = full_r ? 1 : 0;
                 load_info(n + 1);
                 __syncwarp();
                 if (lane == 0) {
@@ -352,8 +360,6 @@ __global__ void __launch_bounds__(384, 1)
             const int bb = n & 1, buf = n % NB;
             const int h = step_h(n), qt = step_qt(n), i0 = qt * BQ;
             const int delta = p.q_off + i0 - j0;
-            const TileBounds tb = p.tile_bounds[size_t(b) * t64 + qt];
-            const bool full = tb.n_nonempty == BQ && tb.max_lo <= j0 && tb.min_hi >= j0 + BK - 1;
             const bool used = band_used(n);
             // warp-uniform waits: S / dP of the step, then its band rows and column info
             if (!warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDkdvS, p.timeout_ns) ||
@@ -376,6 +382,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int u = 0; u < 8; ++u) baddr[u] = band_s + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r);
             const uint32_t info_s = smem_u32(smem + L::INFO_OFF + buf * int(sizeof(StepInfo)));
+            const bool full = lds_s32(info_s + offsetof(StepInfo, full)) != 0;
             // dprofiles[b, h, i0 + c, delta + c - r] for column c = cw + cl: the address of
             // column cl is dbase + cl (R + 1) floats
             char* const dbase = reinterpret_cast<char*>(
