@@ -183,6 +183,14 @@ inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream)
 inkling_status inkling_rel_attn_selftest_wait_timeout(uint32_t timeout_us, void* workspace,
                                                       size_t workspace_bytes, void* stream);
 
+/* Diagnostic: evaluates, on the device, the FMA-pipe power of two the forward
+ * kernel uses for a share of its softmax exponentials (range reduction
+ * t = n + f, a fitted cubic for 2^f, n added to the exponent field):
+ * out[k] = 2^t[k] for k < n, inputs clamped to >= -125. `t` and `out` are device
+ * buffers of n floats owned by the caller. Returns INKLING_ERR_INVALID_ARG for
+ * null pointers or n < 0, INKLING_ERR_CUDA on a launch error; asynchronous. */
+inkling_status inkling_rel_attn_selftest_exp2(const float* t, float* out, int64_t n, void* stream);
+
 /*
  * Diagnostic timing hook. While `events` is non-NULL, each later fwd/bwd call
  * records events[2k] just before and events[2k+1] just after its k-th kernel

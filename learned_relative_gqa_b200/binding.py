@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH):
     lib.inkling_rel_attn_fwd_noalloc.argtypes = [dp] + [vp] * 11 + [vp]
     lib.inkling_rel_attn_last_device_error.restype = ctypes.c_int
     lib.inkling_rel_attn_last_device_error.argtypes = [vp, vp]
+    lib.inkling_rel_attn_selftest_exp2.restype = ctypes.c_int
+    lib.inkling_rel_attn_selftest_exp2.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.inkling_rel_attn_selftest_wait_timeout.restype = ctypes.c_int
     lib.inkling_rel_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
     lib.inkling_rel_attn_set_timing_events.restype = ctypes.c_int
@@ -162,6 +164,12 @@ def inkling_rel_attn_last_device_error(workspace, stream=None) -> int:
 def inkling_rel_attn_selftest_wait_timeout(timeout_us: int, workspace, stream=None) -> int:
     return int(load().inkling_rel_attn_selftest_wait_timeout(int(timeout_us), _p(workspace), workspace.numel(),
                                                              _stream(stream)))
+
+
+def inkling_rel_attn_selftest_exp2(t, out, stream=None) -> None:
+    """t, out: contiguous float32 CUDA tensors of the same size."""
+    _check(load().inkling_rel_attn_selftest_exp2(_p(t), _p(out), int(t.numel()), _stream(stream)),
+           "inkling_rel_attn_selftest_exp2")
 
 
 def inkling_rel_attn_set_timing_events(events, n_pairs: int) -> None:

@@ -40,6 +40,8 @@
 //
 // Operation and argument conventions follow the NeMo AutoModel page for
 // Inkling2FlexAttention.forward; see include/inkling_rel_attn.h.
+#include <type_traits>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -381,6 +383,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 break;
             }
             if (wq == 0 && lane == 0) IRA_TRACE(p, 11 + 3 * s, n);
+            if (s == 0 && lane == 0) IRA_TRACE(p, 28 + wq, n);  // per-warp S ready (head A)
             tc_fence_after();
             uint32_t x[64];
             tmem_ld32(tmem + lane_base + L::s_col(s, buf) + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -403,40 +406,50 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 mx = fmax3(a0, a1, fmaxf(a2, a3));
                 coef = p.scale_log2;
             } else {
-                // x becomes the logit scale * s + profile bias (natural units), masked
-                uint32_t w[33];
-                if (use_band) {
-                    cp_async_wait_group<1>();  // this step's window (the next step's may fly)
-                    const uint32_t* words =
-                        reinterpret_cast<const uint32_t*>(band0 + buf * BAND_BYTES + row_off) + g_r;
+                // x becomes the logit scale * s + profile bias (natural units), masked;
+                // specialised on whether the step reads the band and needs the mask
+                auto pass1 = [&](auto band_c, auto mask_c) {
+                    constexpr bool BAND = decltype(band_c)::value, MASK = decltype(mask_c)::value;
+                    uint32_t w[33];
+                    if (BAND) {
+                        cp_async_wait_group<1>();  // this step's window (the next step's may fly)
+                        if (s == 0 && lane == 0) IRA_TRACE(p, 24 + wq, n);  // per-warp band ready (head A)
+                        const uint32_t* words =
+                            reinterpret_cast<const uint32_t*>(band0 + buf * BAND_BYTES + row_off) + g_r;
 #pragma unroll
-                    for (int q = 0; q < 33; ++q) w[q] = words[q];
-                }
-                const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
-                float a0 = -INFINITY, a1 = -INFINITY;
+                        for (int q = 0; q < 33; ++q) w[q] = words[q];
+                        if (s == 0 && lane == 0) IRA_TRACE(p, 36 + wq, __uint_as_float(w[0]) == 12345.f ? n + 1 : n);
+                    }
+                    // allowed columns [c_lo, c_lo + c_span] (none for an empty row)
+                    const int c_lo = empty ? BN : rb.x - jk, c_span = empty ? 0 : rb.y - rb.x;
+                    float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int pp = 0; pp < 32; ++pp) {
-                    const int c = 2 * pp;
-                    float b0 = 0.f, b1 = 0.f;
-                    if (use_band) {
-                        const uint32_t v = funnel_r(w[31 - pp], w[32 - pp], fshift);
-                        b0 = bf16hi_to_f32(v);  // column c
-                        b1 = bf16lo_to_f32(v);  // column c+1
+                    for (int pp = 0; pp < 32; ++pp) {
+                        const int c = 2 * pp;
+                        float b0 = 0.f, b1 = 0.f;
+                        if (BAND) {
+                            const uint32_t v = funnel_r(w[31 - pp], w[32 - pp], fshift);
+                            b0 = bf16hi_to_f32(v);  // column c
+                            b1 = bf16lo_to_f32(v);  // column c+1
+                        }
+                        float y0 = fmaf(__uint_as_float(x[c]), p.scale, b0);
+                        float y1 = fmaf(__uint_as_float(x[c + 1]), p.scale, b1);
+                        if (MASK) {
+                            y0 = uint32_t(c - c_lo) <= uint32_t(c_span) ? y0 : -INFINITY;
+                            y1 = uint32_t(c + 1 - c_lo) <= uint32_t(c_span) ? y1 : -INFINITY;
+                        }
+                        x[c] = __float_as_uint(y0);
+                        x[c + 1] = __float_as_uint(y1);
+                        a[pp & 3] = fmax3(a[pp & 3], y0, y1);
                     }
-                    float y0 = fmaf(__uint_as_float(x[c]), p.scale, b0);
-                    float y1 = fmaf(__uint_as_float(x[c + 1]), p.scale, b1);
-                    if (need_mask) {
-                        y0 = (c >= c_lo && c <= c_hi) ? y0 : -INFINITY;
-                        y1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? y1 : -INFINITY;
-                    }
-                    x[c] = __float_as_uint(y0);
-                    x[c + 1] = __float_as_uint(y1);
-                    if (pp & 1)
-                        a1 = fmax3(a1, y0, y1);
-                    else
-                        a0 = fmax3(a0, y0, y1);
-                }
-                mx = fmaxf(a0, a1);
+                    if (s == 0 && lane == 0) IRA_TRACE(p, 32 + wq, n);  // per-warp pass-1 math done (head A)
+                    return fmax3(a[0], a[1], fmaxf(a[2], a[3]));
+                };
+                using T_ = std::true_type;
+                using F_ = std::false_type;
+                if (use_band && need_mask) mx = pass1(T_{}, T_{});
+                else if (use_band) mx = pass1(T_{}, F_{});
+                else mx = pass1(F_{}, T_{});
                 coef = kLog2e;
             }
             // this step's band buffer is consumed: fetch the window of step n + 2 into it
@@ -470,7 +483,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     const int c = 32 * q + 2 * u;
                     const float2 t =
                         __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), c2, nb2);
-                    const float2 pr = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    // every second pair on the FMA pipe, the rest on the MUFU
+                    const float2 pr = (u & 1) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
                     pk[u] = pack_bf16x2(pr.x, pr.y);
                     if (u & 1)
                         acc1 = __fadd2_rn(acc1, pr);
@@ -480,6 +494,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 tmem_st16(tmem + lane_base + L::s_col(s, buf) + 16 * q, pk);
             }
             l += (acc0.x + acc0.y) + (acc1.x + acc1.y);
+            if (s == 0 && lane == 0) IRA_TRACE(p, 40 + wq, __float_as_uint(l) == 0x7fffffffu ? n + 1 : n);  // pass 2 issued
 
             // rescale O when a row of this warp moved its maximum; the PV product of
             // step n-1 must be complete first (the one of step n waits for this P).
@@ -502,10 +517,12 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 }
             }
             tmem_wait_st();
+            if (s == 0 && lane == 0) IRA_TRACE(p, 44 + wq, n);  // P in TMEM (head A)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[2 * s + buf]);
             if (wq == 0 && lane == 0) IRA_TRACE(p, 13 + 3 * s, n);
+            if (s == 0 && lane == 0) IRA_TRACE(p, 20 + wq, n);  // per-warp P done (head A)
         }
         cp_async_wait_all();
 

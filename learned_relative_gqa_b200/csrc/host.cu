@@ -439,6 +439,11 @@ inkling_status inkling_rel_attn_selftest_wait_timeout(uint32_t timeout_us, void*
     return inkling_rel_attn_last_device_error(workspace, stream);
 }
 
+inkling_status inkling_rel_attn_selftest_exp2(const float* t, float* out, int64_t n, void* stream) {
+    if (n < 0 || (n > 0 && (!t || !out)) || n > (int64_t(1) << 40)) return INKLING_ERR_INVALID_ARG;
+    return cuda_status(note(launch_selftest_exp2(t, out, n, static_cast<cudaStream_t>(stream))));
+}
+
 inkling_status inkling_rel_attn_set_timing_events(void* const* events, int n_pairs) {
     if (n_pairs < 0) return INKLING_ERR_INVALID_ARG;
     g_events = reinterpret_cast<cudaEvent_t const*>(events);

@@ -21,6 +21,7 @@ cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const flo
 cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
                               cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st);
+cudaError_t launch_selftest_exp2(const float* t, float* out, int64_t n, cudaStream_t st);
 
 // Forward attention. tm_q: {D, Hq, S, B} box {64,1,128,1}; tm_k / tm_v: {D, Hkv, Skv, B} box {64,1,64,1}.
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,

@@ -281,6 +281,15 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, int* err) {
     __syncthreads();
 }
 
+// Device evaluation of exp2_fma2 (the forward's FMA-pipe power of two), for its accuracy test.
+__global__ void selftest_exp2_kernel(const float* __restrict__ t, float* __restrict__ out, int64_t n) {
+    const int64_t k = 2 * (int64_t(blockIdx.x) * blockDim.x + threadIdx.x);
+    if (k >= n) return;
+    const float2 v = exp2_fma2(make_float2(t[k], k + 1 < n ? t[k + 1] : 0.f));
+    out[k] = v.x;
+    if (k + 1 < n) out[k + 1] = v.y;
+}
+
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
@@ -328,6 +337,13 @@ cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int 
     if (rows == 0 || R == 0) return cudaSuccess;
     const int blocks = int(rows / 8 + 1 < 148 * 32 ? rows / 8 + 1 : 148 * 32);
     dprof_zero_kernel<<<blocks, 256, 0, st>>>(row_bounds, B, S, Hq, R, q_off, dprof);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_exp2(const float* t, float* out, int64_t n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = ((n + 1) / 2 + 255) / 256;
+    selftest_exp2_kernel<<<unsigned(blocks), 256, 0, st>>>(t, out, n);
     return cudaGetLastError();
 }
 

@@ -299,6 +299,30 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^t for two values on the FMA and integer pipes, so that a share of the softmax
+// exponentials leaves the MUFU (which also performs the BF16 conversions) free.
+// Method: Cody-Waite style range reduction t = n + f with n = round(t) obtained by
+// adding and subtracting 1.5 * 2^23 (round-to-nearest in FP32), f in [-1/2, 1/2];
+// 2^f from a cubic fitted here to 2^f on that interval (weighted least squares towards
+// minimax relative error; max relative error 7.6e-5 when evaluated in FP32 by Horner's
+// rule); n is then added to the exponent field. Inputs are clamped to >= -125 so the
+// exponent stays in range (results below 2^-125 come out as about 2^-125, not 0); the
+// callers' arguments never exceed +9.
+__device__ __forceinline__ float2 exp2_fma2(float2 t) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999282360076904f, c1 = 0.6932609677314758f, c2 = 0.24260851740837097f,
+                    c3 = 0.05517049878835678f;
+    t = make_float2(fmaxf(t.x, -125.f), fmaxf(t.y, -125.f));
+    const float2 r = __fadd2_rn(t, make_float2(kRound, kRound));         // n in the low mantissa bits
+    const float2 nf = __fadd2_rn(r, make_float2(-kRound, -kRound));      // n as a float
+    const float2 f = __ffma2_rn(nf, make_float2(-1.f, -1.f), t);          // t - n
+    float2 q = __ffma2_rn(f, make_float2(c3, c3), make_float2(c2, c2));
+    q = __ffma2_rn(q, f, make_float2(c1, c1));
+    q = __ffma2_rn(q, f, make_float2(c0, c0));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(r.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(r.y) << 23)));
+}
+
 // max of three floats (single sm_100 instruction)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
