@@ -530,11 +530,14 @@ def main():
         for _ in range(2):
             bl.fwd()
         torch.cuda.synchronize()
+        sampler_l = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_long_rank{rank}.csv")) \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, f"/tmp/clocks_long_rank{rank}.csv")
         ms_l = timed(bl.fwd, args.long_steps, torch.cuda.synchronize) / args.long_steps
+        clocks_l = sampler_l.stop()
         tfl = 4.0 * wl.head_dim * El / (ms_l * 1e-3) / 1e12
         long_fwd = {"workload": "long: B1 S32768 Hq32 Hkv8 D128 R4096 full causal", "ms": round(ms_l, 3),
                     "allowed_elements": El, "tflops": round(tfl, 1),
-                    "pct_of_bf16_peak": round(100 * tfl / peaks["bf16_tflops"], 1)}
+                    "pct_of_bf16_peak": round(100 * tfl / peaks["bf16_tflops"], 1), "clocks": clocks_l}
         del bl, xl
         torch.cuda.empty_cache()
 
