@@ -538,7 +538,9 @@ constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
 constexpr int BAND_BYTES = BAND_UNITS * 16;
 constexpr int QTILE = BM * 128;       // [128 x 64 bf16]
 constexpr int KTILE = BN * 128;       // [64 x 64 bf16]
-constexpr int NST = 3;                // K / V stages (two steps of lookahead)
+constexpr int NSB = 3;                // S / dP buffers in TMEM: the MMAs run two steps ahead
+constexpr int NSK = 4;                // K stages: K(n) is read by S(n) and, two steps later, by dQ(n)
+constexpr int NSV = 2;                // V stages: V(n) is read by dP(n) only
 
 __host__ __device__ constexpr int band_unit(int r) { return BAND_CHUNKS * r + 2 * (r >> 3); }
 
@@ -547,12 +549,13 @@ struct Layout {
     static constexpr int KB = D / 64;
     static constexpr int Q_OFF = 0;
     static constexpr int DO_OFF = Q_OFF + KB * QTILE;
-    static constexpr int K_OFF = DO_OFF + KB * QTILE;          // NST stages
-    static constexpr int V_OFF = K_OFF + NST * KB * KTILE;     // NST stages
-    static constexpr int BAND_OFF = V_OFF + NST * KB * KTILE;  // [warpgroup][step parity]
+    static constexpr int K_OFF = DO_OFF + KB * QTILE;          // NSK stages
+    static constexpr int V_OFF = K_OFF + NSK * KB * KTILE;     // NSV stages
+    static constexpr int BAND_OFF = V_OFF + NSV * KB * KTILE;  // [warpgroup][step parity]
     static constexpr int BAR_OFF = BAND_OFF + 4 * BAND_BYTES;
-    // q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], acc_full, drain
-    static constexpr int NBARS = 7 + 2 * NST;
+    // q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[NSB], p_full[NSB],
+    // acc_full, drain
+    static constexpr int NBARS = 3 + 2 * NSK + 2 * NSV + 2 * NSB;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -569,19 +572,21 @@ __global__ void __launch_bounds__(384, 1)
               const AttnParams p, const int num_qtiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9, MMA_WARP_B = 11;
+    constexpr int TMA_WARP = 8, MMA_WARP = 9, V_WARP = 10, MMA_WARP_B = 11;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
-    uint64_t* kv_full = bars + 1;              // [NST]
-    uint64_t* kv_empty = bars + 1 + NST;       // [NST]
-    uint64_t* s_full = bars + 1 + 2 * NST;     // [2]
-    uint64_t* p_full = bars + 3 + 2 * NST;     // [2]
-    uint64_t* acc_full = bars + 5 + 2 * NST;
-    uint64_t* drain = bars + 6 + 2 * NST;
+    uint64_t* k_full = bars + 1;               // [NSK]
+    uint64_t* k_empty = k_full + NSK;          // [NSK]
+    uint64_t* v_full = k_empty + NSK;          // [NSV]
+    uint64_t* v_empty = v_full + NSV;          // [NSV]
+    uint64_t* s_full = v_empty + NSV;          // [NSB]
+    uint64_t* p_full = s_full + NSB;           // [NSB]
+    uint64_t* acc_full = p_full + NSB;
+    uint64_t* drain = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -599,11 +604,17 @@ __global__ void __launch_bounds__(384, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         // a K / V stage is free, and S / dP of a step ready, once both MMA issuers committed
-        for (int u = 0; u < NST; ++u) {
-            mbar_init(&kv_full[u], 1);
-            mbar_init(&kv_empty[u], 2);
+        // a K stage is free once S (issuer A) and dQ (issuer B) of its step completed,
+        // a V stage once dP (issuer B) did
+        for (int u = 0; u < NSK; ++u) {
+            mbar_init(&k_full[u], 1);
+            mbar_init(&k_empty[u], 2);
         }
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < NSV; ++u) {
+            mbar_init(&v_full[u], 1);
+            mbar_init(&v_empty[u], 1);
+        }
+        for (int u = 0; u < NSB; ++u) {
             mbar_init(&s_full[u], 2);
             mbar_init(&p_full[u], 8);
         }
@@ -641,8 +652,8 @@ __global__ void __launch_bounds__(384, 1)
 
     auto q_smem = [&](int kb) { return smem + L::Q_OFF + kb * QTILE; };
     auto do_smem = [&](int kb) { return smem + L::DO_OFF + kb * QTILE; };
-    auto k_smem = [&](int st, int kb) { return smem + L::K_OFF + (st * KB + kb) * KTILE; };
-    auto v_smem = [&](int st, int kb) { return smem + L::V_OFF + (st * KB + kb) * KTILE; };
+    auto k_smem = [&](int n, int kb) { return smem + L::K_OFF + ((n % NSK) * KB + kb) * KTILE; };
+    auto v_smem = [&](int n, int kb) { return smem + L::V_OFF + ((n % NSV) * KB + kb) * KTILE; };
     auto key0 = [&](int n) { return i0g + BN - (t_begin + n) * BN; };
 
     // Launched with 384 x 168 registers; warpgroup 2 (producer, two MMA issuers, an idle
@@ -650,49 +661,64 @@ __global__ void __launch_bounds__(384, 1)
     // (128 x 80 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
     if (warp >= 8) {
         setmaxnreg_dec<80>();
-    if (warp == TMA_WARP) {
+    if (warp == TMA_WARP || warp == V_WARP) {
+        // ------------------------------------------------------------ tile producers:
+        // Q and dO once plus the K ring (TMA_WARP), the V ring (V_WARP)
+        const bool is_v = warp == V_WARP;
         if (lane == 0 && n_steps > 0) {
-            prefetch_tensormap(&tm_q);
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
-            prefetch_tensormap(&tm_do);
-            mbar_arrive_expect_tx(q_full, 2 * KB * QTILE);
-            for (int kb = 0; kb < KB; ++kb) {
-                tma_load_4d(q_smem(kb), &tm_q, q_full, kb * 64, h, i0, b);
-                tma_load_4d(do_smem(kb), &tm_do, q_full, kb * 64, h, i0, b);
+            if (!is_v) {
+                prefetch_tensormap(&tm_q);
+                prefetch_tensormap(&tm_do);
+                prefetch_tensormap(&tm_k);
+                mbar_arrive_expect_tx(q_full, 2 * KB * QTILE);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_4d(q_smem(kb), &tm_q, q_full, kb * 64, h, i0, b);
+                    tma_load_4d(do_smem(kb), &tm_do, q_full, kb * 64, h, i0, b);
+                }
+            } else {
+                prefetch_tensormap(&tm_v);
             }
+            const int ns = is_v ? NSV : NSK;
+            uint64_t* full = is_v ? v_full : k_full;
+            uint64_t* empty = is_v ? v_empty : k_empty;
             int last = -1;
             for (int n = 0; n < n_steps; ++n) {
-                const int st = n % NST;
-                if (!mbar_wait(&kv_empty[st], ((n / NST) & 1) ^ 1, ctl, p.err, kErrDqKVFree, p.timeout_ns)) break;
-                const int jk = key0(n);
-                mbar_arrive_expect_tx(&kv_full[st], 2 * KB * KTILE);
+                const int st = n % ns;
+                if (!mbar_wait(&empty[st], ((n / ns) & 1) ^ 1, ctl, p.err, kErrDqKVFree, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&full[st], KB * KTILE);
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_4d(k_smem(st, kb), &tm_k, &kv_full[st], kb * 64, g, jk, b);
-                    tma_load_4d(v_smem(st, kb), &tm_v, &kv_full[st], kb * 64, g, jk, b);
+                    if (is_v)
+                        tma_load_4d(v_smem(n, kb), &tm_v, &full[st], kb * 64, g, key0(n), b);
+                    else
+                        tma_load_4d(k_smem(n, kb), &tm_k, &full[st], kb * 64, g, key0(n), b);
                 }
-                IRA_TRACE(p, 41, n);
+                if (!is_v) IRA_TRACE(p, 41, n);
                 last = n;
             }
-            mbar_wait_drain(q_full, 0, p.timeout_ns);
-            for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
-                mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.timeout_ns);
+            if (!is_v) mbar_wait_drain(q_full, 0, p.timeout_ns);
+            for (int n = (last >= ns ? last - ns + 1 : 0); n <= last; ++n)
+                mbar_wait_drain(&full[n % ns], (n / ns) & 1, p.timeout_ns);
         }
     } else if (warp == MMA_WARP || warp == MMA_WARP_B) {
         // ------------------------------------------------------------ MMA issuers
         // Two issuing threads so that one's waits never starve the tensor core:
-        // A issues S = Q K^T; B issues dP = dO V^T and dQ += dS K (dS from TMEM). Each
-        // overwrites its S / dP buffer only after the elementwise warps are done with the
-        // step that used it, and B's dQ of that step precedes it in B's issue order.
+        // A issues S = Q K^T; B issues dP = dO V^T and dQ += dS K (dS from TMEM). With
+        // three S / dP buffers the scores of step n + 2 are issued while the elementwise
+        // warps work on step n + 1. Each issuer overwrites a buffer only after the
+        // elementwise warps are done with the step that used it, and B's dQ of that
+        // step precedes it in B's issue order.
         const bool is_b = warp == MMA_WARP_B;
         if (lane == 0 && n_steps > 0) {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
             constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t a_base = smem_u32(is_b ? do_smem(0) : q_smem(0));
-            auto b_base = [&](int st) { return smem_u32(is_b ? v_smem(st, 0) : k_smem(st, 0)); };
+            auto wait_tile = [&](int n) {  // K(n) for A, V(n) for B
+                return is_b ? mbar_wait(&v_full[n % NSV], (n / NSV) & 1, ctl, p.err, kErrDqKV, p.timeout_ns)
+                            : mbar_wait(&k_full[n % NSK], (n / NSK) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
+            };
             auto issue_score = [&](int n) {  // S (A) or dP (B) of step n
-                const int st = n % NST, bb = n & 1;
-                const uint32_t bs = b_base(st);
+                const int bb = n % NSB;
+                const uint32_t bs = smem_u32(is_b ? v_smem(n, 0) : k_smem(n, 0));
                 const uint32_t col = is_b ? L::dp_col(bb) : L::s_col(bb);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -702,31 +728,39 @@ __global__ void __launch_bounds__(384, 1)
                            kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[bb]);
-                // A's last read of this K stage
-                if (!is_b) mma_commit(&kv_empty[st]);
+                // last read of V(n) by B; A's read of K(n)
+                mma_commit(is_b ? &v_empty[n % NSV] : &k_empty[n % NSK]);
                 if (!is_b) IRA_TRACE(p, 42, n);
             };
-            bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns) &&
-                      mbar_wait(&kv_full[0], 0, ctl, p.err, kErrDqKV, p.timeout_ns);
-            if (ok) {
+            bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns);
+            for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
+                ok = wait_tile(n);
+                if (!ok) break;
                 tc_fence_after();
-                issue_score(0);
+                issue_score(n);
             }
             for (int n = 0; ok && n < n_steps; ++n) {
-                if (n + 1 < n_steps) {
-                    ok = mbar_wait(&kv_full[(n + 1) % NST], ((n + 1) / NST) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
+                // S / dP of step n + 2 go into the buffer of step n - 1, free once the
+                // elementwise warps are done with it (P(n-1), awaited last iteration)
+                // and, for B, behind dQ(n-1) in issue order
+                if (n + 2 < n_steps) {
+                    ok = wait_tile(n + 2);
                     if (!ok) break;
-                    if (!is_b) IRA_TRACE(p, 49, n + 1);
+                    if (!is_b) IRA_TRACE(p, 49, n + 2);
                     tc_fence_after();
-                    issue_score(n + 1);
+                    issue_score(n + 2);
                 }
-                ok = mbar_wait(&p_full[n & 1], (n >> 1) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
+                ok = mbar_wait(&p_full[n % NSB], (n / NSB) & 1, ctl, p.err, kErrDqP, p.timeout_ns);
                 if (!ok) break;
                 if (!is_b) continue;
+                // K(n) arrived long ago (A issued S(n) on it); B takes the same phase
+                // for its own ordering with the copy
+                ok = mbar_wait(&k_full[n % NSK], (n / NSK) & 1, ctl, p.err, kErrDqKV, p.timeout_ns);
+                if (!ok) break;
                 IRA_TRACE(p, 43, n);
                 tc_fence_after();
-                const int st = n % NST, bb = n & 1;
-                const uint32_t ks = smem_u32(k_smem(st, 0));
+                const int bb = n % NSB;
+                const uint32_t ks = smem_u32(k_smem(n, 0));
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     // dS of key columns [32 w, 32 w + 32) sits, packed, at the start of
@@ -734,7 +768,7 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + HALF * (kk >> 1) + 8 * (kk & 1),
                            sdesc_sw128(ks + kk * 2048, KTILE, 1024), IDESC_DQ, (n > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&kv_empty[st]);
+                mma_commit(&k_empty[n % NSK]);
                 IRA_TRACE(p, 44, n);
             }
             if (ok && is_b) mma_commit(acc_full);
@@ -797,12 +831,12 @@ __global__ void __launch_bounds__(384, 1)
         const float2 nl2 = make_float2(-lse2, -lse2);
         const float2 nv2 = make_float2(-dvr, -dvr);
         for (int n = 0; n < n_steps; ++n) {
-            const int bb = n & 1;
+            const int bb = n % NSB;
             const int jk = key0(n) + cw;  // key of this warpgroup's first column
             const bool my_full = empty || (rb.x <= jk && rb.y >= jk + HALF - 1);
             const bool need_mask = !__all_sync(0xffffffffu, my_full);
             const bool use_band = band_needed(n);
-            if (!warp_wait(&s_full[bb], (n >> 1) & 1, ctl, p.err, kErrDqS, p.timeout_ns)) {
+            if (!warp_wait(&s_full[bb], (n / NSB) & 1, ctl, p.err, kErrDqS, p.timeout_ns)) {
                 ok = false;
                 break;
             }
@@ -815,7 +849,7 @@ __global__ void __launch_bounds__(384, 1)
             if (use_band) {
                 cp_async_wait_group<1>();  // this step's window (the next step's may fly)
                 const uint32_t* words =
-                    reinterpret_cast<const uint32_t*>(smem + L::BAND_OFF + (2 * w + bb) * BAND_BYTES + unit * 16) + g_r;
+                    reinterpret_cast<const uint32_t*>(smem + L::BAND_OFF + (2 * w + (n & 1)) * BAND_BYTES + unit * 16) + g_r;
 #pragma unroll
                 for (int q = 0; q < 17; ++q) wv[q] = words[q];
             }
