@@ -550,11 +550,7 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": (f"{w.name}: B{w.batch} S{w.seq} Hq{w.heads_q} Hkv{w.heads_kv} D{w.head_dim} "
-                                    f"W{w.window} R{w.rel_extent} docs{w.docs} pad{w.pad}, fwd+bwd"),
-                       "global_batch": w.batch * world, "seq_len": w.seq, "parallelism": f"replicas x{world}",
-                       "allowed_elements": E, "flops_per_step": flops_step,
-                       "l2": "inputs larger than L2 (profiles %.2f GB/step)" % (x["profiles"].numel() * 2 / 1e9)},
+            "config": run_config(w, x, E, flops_step, world),
             "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
             "roofline": roof, "kernels": kernels, "gpu_launches": gpu_launches,
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks, "long_fwd": long_fwd,
@@ -565,12 +561,22 @@ def main():
         dist.destroy_process_group()
 
 
+def run_config(w, x, E, flops_step, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": (f"{w.name}: B{w.batch} S{w.seq} Hq{w.heads_q} Hkv{w.heads_kv} D{w.head_dim} "
+                         f"W{w.window} R{w.rel_extent} docs{w.docs} pad{w.pad}, {'fwd+bwd' if w.backward else 'fwd'}"),
+            "global_batch": w.batch * world, "seq_len": w.seq, "parallelism": f"replicas x{world}",
+            "allowed_elements": E, "flops_per_step": flops_step,
+            "l2": "inputs larger than L2 (profiles %.2f GB/step)" % (x["profiles"].numel() * 2 / 1e9)}
+
+
 def run_reference(args, w, backward):
     """The oracle as the reference arm: each step is the FP64 oracle forward+backward
     on a bounded sample of the same workload, on the host cores."""
     from learned_relative_gqa_b200 import workloads
     x = workloads.make_inputs(w, "cpu")
     D = w.head_dim
+    E_full = workloads.allowed_counts(w, x)
     s_sub, hc, E, dt = calibrate_sample(x, target_s=4.0, max_s=15.0)
     for _ in range(min(args.warmup, 1)):
         oracle_sample_step(hc)
@@ -586,8 +592,7 @@ def run_reference(args, w, backward):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": (f"{w.name}: B{w.batch} S{w.seq} Hq{w.heads_q} Hkv{w.heads_kv} D{w.head_dim} "
-                                f"W{w.window} R{w.rel_extent} docs{w.docs}, fwd+bwd (oracle sample)")},
+        "config": run_config(w, x, E_full, (14.0 if backward else 4.0) * D * E_full, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
