@@ -74,6 +74,9 @@ typedef enum {
  *   rel_extent   R     width of each profiles row, a multiple of 8 (0 allowed)
  *   window       W     sliding window (keys with i_g - j < W); 0 = full causal
  *   query_offset       global column of local query row 0; 0 without CP
+ * Size limits (INKLING_ERR_UNSUPPORTED beyond them): S, Skv, query_offset, B, R,
+ * W < 2^30; Hq < 65536; the tile grids below 2^31 CTAs; and, when R > 0,
+ * B * Hq * S below 2^31 - 256 (the backward addresses profile rows as int32).
  */
 typedef struct {
     int64_t batch, seq_q, seq_k, heads_q, heads_kv, head_dim, rel_extent, window, query_offset;

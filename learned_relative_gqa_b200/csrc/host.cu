@@ -122,6 +122,9 @@ inkling_status check_dims(const inkling_rel_attn_dims* d) {
     const int64_t nqt = (d->seq_q + 127) / 128, nkt = (d->seq_k + 127) / 128;
     if (nqt * d->batch * d->heads_q >= (int64_t(1) << 31) || nkt * d->batch * d->heads_kv >= (int64_t(1) << 31))
         return INKLING_ERR_UNSUPPORTED;
+    // the backward's profile-band tensor copies address profile rows b * Hq * S + h * S + i as one int32
+    if (d->rel_extent > 0 && d->batch * d->heads_q * d->seq_q >= (int64_t(1) << 31) - 256)
+        return INKLING_ERR_UNSUPPORTED;
     return INKLING_OK;
 }
 

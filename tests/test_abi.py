@@ -69,6 +69,8 @@ def test_workspace_size(lib):
     (dict(heads_q=6, heads_kv=4), 1),
     (dict(window=-1), 1),
     (dict(seq_q=-3), 1),
+    # profile rows b * Hq * S + h * S + i must stay below 2^31 when R > 0
+    (dict(batch=64, heads_q=64, heads_kv=8, seq_q=1 << 19, seq_k=1 << 19), 2),
 ])
 def test_fwd_rejects_bad_dims_on_host(lib, bad, expect):
     d = dims(**bad)
