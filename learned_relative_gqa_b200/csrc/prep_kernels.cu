@@ -234,32 +234,41 @@ __global__ void bwd_prep_kernel(const float* __restrict__ out, const float* __re
 
 // Zero the dprofiles entries of each (b, h, i) row that no allowed key
 // reaches: everything outside the visited distances [i_g - hi, i_g - lo].
-// One warp per row.
+// One warp per 32 consecutive rows of one (b, h): lane l reads the bounds of row
+// i0 + l, then the warp zeroes row by row (bounds broadcast by shuffles, 16-byte
+// stores, rows the attention kernels cover entirely skipped).
 __global__ void dprof_zero_kernel(const int2* __restrict__ row_bounds, int B, int S, int Hq, int R, int q_off,
                                   float* __restrict__ dprof) {
-    const int64_t nrows = int64_t(B) * Hq * S;
     const int lane = threadIdx.x & 31;
-    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t row = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows; row += warps) {
-        const int i = int(row % S);
-        const int b = int(row / (int64_t(S) * Hq));
-        const int2 bh = row_bounds[size_t(b) * S + i];
-        const int ig = q_off + i;
-        int dlo = R, dhi = -1;  // visited distances (inclusive); empty by default
-        if (bh.x <= bh.y) {
-            dlo = max(0, ig - bh.y);
-            dhi = min(R - 1, ig - bh.x);
+    const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    const int segs = (S + 31) >> 5;  // 32-row segments per (b, h)
+    const int64_t nseg = int64_t(B) * Hq * segs;
+    for (int64_t sg = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; sg < nseg; sg += nwarps) {
+        const int64_t bh = sg / segs;
+        const int i0 = int(sg - bh * segs) * 32;
+        const int b = int(bh / Hq);
+        int dlo_l = R, dhi_l = -1;  // visited distances of row i0 + lane (inclusive); none by default
+        const int il = i0 + lane;
+        if (il < S) {
+            const int2 bnd = row_bounds[size_t(b) * S + il];
+            if (bnd.x <= bnd.y) {
+                dlo_l = max(0, q_off + il - bnd.y);
+                dhi_l = min(R - 1, q_off + il - bnd.x);
+            }
         }
-        float* base = dprof + row * int64_t(R);
-        for (int e0 = lane * 4; e0 < R; e0 += 128) {
-            const bool all_out = (e0 + 3 < dlo) || (e0 > dhi);
-            if (all_out) {
-                *reinterpret_cast<float4*>(base + e0) = make_float4(0.f, 0.f, 0.f, 0.f);
-            } else {
+        const int nrows = min(32, S - i0);
+        for (int r = 0; r < nrows; ++r) {
+            const int dlo = __shfl_sync(0xffffffffu, dlo_l, r);
+            const int dhi = __shfl_sync(0xffffffffu, dhi_l, r);
+            if (dlo == 0 && dhi == R - 1) continue;
+            float* base = dprof + (bh * S + i0 + r) * int64_t(R);
+            for (int e0 = lane * 4; e0 < R; e0 += 128) {
+                if (e0 + 3 < dlo || e0 > dhi) {
+                    *reinterpret_cast<float4*>(base + e0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (e0 < dlo || e0 + 3 > dhi) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = e0 + u;
-                    if (e < dlo || e > dhi) base[e] = 0.f;
+                    for (int u = 0; u < 4; ++u)
+                        if (e0 + u < dlo || e0 + u > dhi) base[e0 + u] = 0.f;
                 }
             }
         }
@@ -333,9 +342,10 @@ cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const flo
 
 cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
                               cudaStream_t st) {
-    const long long rows = (long long)B * S * Hq;
-    if (rows == 0 || R == 0) return cudaSuccess;
-    const int blocks = int(rows / 8 + 1 < 148 * 32 ? rows / 8 + 1 : 148 * 32);
+    const long long segs = (long long)B * Hq * ((S + 31) / 32);
+    if (segs == 0 || R == 0) return cudaSuccess;
+    const long long want = (segs + 7) / 8;  // 8 warps per block
+    const int blocks = int(want < 148 * 16 ? want : 148 * 16);
     dprof_zero_kernel<<<blocks, 256, 0, st>>>(row_bounds, B, S, Hq, R, q_off, dprof);
     return cudaGetLastError();
 }
