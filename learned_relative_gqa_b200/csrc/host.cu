@@ -104,7 +104,36 @@ struct LaunchTimer {
         ++k;
         return e;
     }
+    bool active() const { return g_events != nullptr; }
 };
+
+// Per host thread and device: a second stream and two events, so that the dK/dV and
+// dQ kernels of one backward call can run side by side (each fills the other's last,
+// partial wave of CTAs). Fork: the side stream waits for the caller's stream; join:
+// the caller's stream waits for the side stream. Works under stream capture.
+struct SideStream {
+    int device = -1;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, ready = nullptr, join = nullptr;
+};
+cudaError_t side_stream(SideStream** out) {
+    thread_local SideStream per_dev[16];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+    SideStream& r = per_dev[dev];
+    if (r.s == nullptr) {
+        e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.ready, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        r.device = dev;
+    }
+    *out = &r;
+    return cudaSuccess;
+}
 
 inkling_status check_dims(const inkling_rel_attn_dims* d) {
     if (!d) return INKLING_ERR_INVALID_ARG;
@@ -373,18 +402,21 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     LaunchTimer tm(st);
     s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
     if (s != INKLING_OK) return s;
-    cudaError_t e = tm.run([&] {
-        return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
-                               lse2t, dvt, st);
-    });
-    if (e == cudaSuccess)
-        e = tm.run([&] {
-            return dims->rel_extent > 0 ? launch_dprof_zero(w.row_bounds(), int(B), int(S), int(Hq),
-                                                            int(dims->rel_extent), int(dims->query_offset),
-                                                            dprofiles, st)
-                                        : cudaSuccess;
-        });
-    if (e != cudaSuccess) return INKLING_ERR_CUDA;
+    // Two streams, except while the timing hook is on (it wants one kernel at a time):
+    //   caller's stream: prep -> dK/dV
+    //   side stream:     dprofiles zeroing (needs only the row bounds) -> wait prep -> dQ
+    // dK/dV and dQ read the same inputs and write disjoint outputs; the zeroing writes the
+    // dprofiles entries that dK/dV does not (distances outside a row's visited range).
+    SideStream* side = nullptr;
+    const bool overlap = !tm.active();
+    cudaError_t e = cudaSuccess;
+    if (overlap) {
+        e = side_stream(&side);
+        if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    cudaStream_t st2 = overlap ? side->s : st;
     AttnParams p = base_params(dims, w, profiles, sink);
     p.lse2t = lse2t;
     p.dvt = dvt;
@@ -392,9 +424,28 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     p.dk = dk;
     p.dv = dv;
     p.dprofiles = dprofiles;
-    e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, tband, p, st) : cudaSuccess; });
-    if (e != cudaSuccess) return INKLING_ERR_CUDA;
-    return cuda_status(tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st); }));
+    e = tm.run([&] {
+        return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
+                               lse2t, dvt, st);
+    });
+    if (e == cudaSuccess && overlap) e = cudaEventRecord(side->ready, st);
+    if (e == cudaSuccess)
+        e = tm.run([&] {
+            return dims->rel_extent > 0 ? launch_dprof_zero(w.row_bounds(), int(B), int(S), int(Hq),
+                                                            int(dims->rel_extent), int(dims->query_offset),
+                                                            dprofiles, st2)
+                                        : cudaSuccess;
+        });
+    if (e == cudaSuccess)
+        e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, tband, p, st) : cudaSuccess; });
+    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st2, side->ready, 0);
+    if (e == cudaSuccess) e = tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st2); });
+    if (overlap) {  // join, on the error paths too, so that no work stays forked off the caller's stream
+        cudaError_t e2 = cudaEventRecord(side->join, side->s);
+        if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, side->join, 0);
+        if (e == cudaSuccess) e = e2;
+    }
+    return cuda_status(e);
 }
 
 inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
