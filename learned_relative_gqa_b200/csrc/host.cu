@@ -114,7 +114,7 @@ struct LaunchTimer {
 struct SideStream {
     int device = -1;
     cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, ready = nullptr, join = nullptr;
+    cudaEvent_t fork = nullptr, bounds = nullptr, ready = nullptr, join = nullptr;
 };
 cudaError_t side_stream(SideStream** out) {
     thread_local SideStream per_dev[16];
@@ -126,6 +126,7 @@ cudaError_t side_stream(SideStream** out) {
     if (r.s == nullptr) {
         e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.bounds, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.ready, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming);
         if (e != cudaSuccess) return e;
@@ -400,11 +401,9 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     if (dims->rel_extent > 0 && !encode_band(&tband, profiles, B * Hq * S, dims->rel_extent)) return INKLING_ERR_CUDA;
 
     LaunchTimer tm(st);
-    s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
-    if (s != INKLING_OK) return s;
     // Two streams, except while the timing hook is on (it wants one kernel at a time):
-    //   caller's stream: prep -> dK/dV
-    //   side stream:     dprofiles zeroing (needs only the row bounds) -> wait prep -> dQ
+    //   caller's stream: prep -> (wait row bounds) -> dK/dV
+    //   side stream:     key span, row bounds -> dprofiles zeroing -> (wait prep) -> dQ
     // dK/dV and dQ read the same inputs and write disjoint outputs; the zeroing writes the
     // dprofiles entries that dK/dV does not (distances outside a row's visited range).
     SideStream* side = nullptr;
@@ -417,6 +416,17 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
         if (e != cudaSuccess) return cuda_status(e);
     }
     cudaStream_t st2 = overlap ? side->s : st;
+    auto join = [&](inkling_status r) {  // on the error paths too: no work stays forked off
+        if (overlap) {
+            cudaError_t e2 = cudaEventRecord(side->join, side->s);
+            if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, side->join, 0);
+            if (r == INKLING_OK && e2 != cudaSuccess) r = cuda_status(e2);
+        }
+        return r;
+    };
+    s = run_bounds(dims, w, valid, key_valid, positions, st2, tm);
+    if (s != INKLING_OK) return join(s);
+    if (overlap) e = cudaEventRecord(side->bounds, st2);
     AttnParams p = base_params(dims, w, profiles, sink);
     p.lse2t = lse2t;
     p.dvt = dvt;
@@ -424,10 +434,11 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     p.dk = dk;
     p.dv = dv;
     p.dprofiles = dprofiles;
-    e = tm.run([&] {
-        return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
-                               lse2t, dvt, st);
-    });
+    if (e == cudaSuccess)
+        e = tm.run([&] {
+            return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
+                                   lse2t, dvt, st);
+        });
     if (e == cudaSuccess && overlap) e = cudaEventRecord(side->ready, st);
     if (e == cudaSuccess)
         e = tm.run([&] {
@@ -436,16 +447,12 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
                                                             dprofiles, st2)
                                         : cudaSuccess;
         });
+    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st, side->bounds, 0);
     if (e == cudaSuccess)
         e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, tband, p, st) : cudaSuccess; });
     if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st2, side->ready, 0);
     if (e == cudaSuccess) e = tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st2); });
-    if (overlap) {  // join, on the error paths too, so that no work stays forked off the caller's stream
-        cudaError_t e2 = cudaEventRecord(side->join, side->s);
-        if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, side->join, 0);
-        if (e == cudaSuccess) e = e2;
-    }
-    return cuda_status(e);
+    return join(cuda_status(e));
 }
 
 inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,

@@ -41,12 +41,34 @@ __device__ __forceinline__ int warp_sum(int v) {
 
 }  // namespace
 
-// grid (B), block 256
+// Bit 7 of each byte of the result is set where that byte of x is nonzero.
+__device__ __forceinline__ uint32_t nonzero_bytes(uint32_t x) {
+    return (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x) & 0x80808080u;
+}
+
+// grid (B), block 512. Rows whose start is 16-byte aligned are read 16 bytes per
+// thread and load (the whole row of a 8192-key batch in one round trip); the
+// rest of a row (and unaligned rows) byte by byte.
 __global__ void kspan_kernel(const uint8_t* __restrict__ key_valid, int Skv, int2* __restrict__ kspan) {
     const int b = blockIdx.x;
+    const uint8_t* row = key_valid + size_t(b) * Skv;
     int first = 0x7FFFFFFF, last = -1;
-    for (int j = threadIdx.x; j < Skv; j += blockDim.x) {
-        if (key_valid[size_t(b) * Skv + j]) {
+    const int vec_end = (reinterpret_cast<uintptr_t>(row) & 15) == 0 ? (Skv & ~15) : 0;
+#pragma unroll 4
+    for (int j0 = threadIdx.x * 16; j0 < vec_end; j0 += blockDim.x * 16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + j0));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t m = nonzero_bytes(w[u]);
+            if (m) {  // little endian: byte t of the word is bits 8t..8t+7
+                first = min(first, j0 + 4 * u + ((__ffs(int(m)) - 1) >> 3));
+                last = max(last, j0 + 4 * u + ((31 - __clz(int(m))) >> 3));
+            }
+        }
+    }
+    for (int j = vec_end + threadIdx.x; j < Skv; j += blockDim.x) {
+        if (row[j]) {
             first = min(first, j);
             last = max(last, j);
         }
@@ -304,7 +326,7 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ t, float* __restr
 // ---------------------------------------------------------------------------
 cudaError_t launch_kspan(const uint8_t* key_valid, int B, int Skv, int2* kspan, cudaStream_t st) {
     if (B == 0) return cudaSuccess;
-    kspan_kernel<<<B, 256, 0, st>>>(key_valid, Skv, kspan);
+    kspan_kernel<<<B, 512, 0, st>>>(key_valid, Skv, kspan);
     return cudaGetLastError();
 }
 

@@ -114,3 +114,21 @@ def test_forward_default_masks_and_positions():
     o_ref, l_ref, _ = oracle.forward(h["q"], h["k"], h["v"], h["profiles"], h["sink"], h["valid"], window=64)
     U.assert_out_close(out.cpu().numpy(), o_ref)
     U.assert_lse_close(lse.cpu().numpy(), l_ref)
+
+
+@pytest.mark.parametrize("seq_k", [523, 512])
+def test_forward_key_span_starts_and_ends_inside_words(seq_k):
+    """Key streams whose valid span starts at column 0, 5, 16 or 37 and ends at a
+    random column, with rows that start on and off 16-byte boundaries: the key span
+    (first / last valid key of each batch row) is found for every alignment."""
+    from learned_relative_gqa_b200 import binding
+    w = U.custom(f"kspan_{seq_k}", 4, 200, 4, 2, 64, 0, 64, docs=(40, 180), pad=(0, 20), seq_k=seq_k,
+                 query_offset=seq_k - 223)
+    x = W.make_inputs(w, "cuda")
+    for b, a in enumerate((0, 5, 16, 37)):
+        x["key_valid"][b, :a] = False
+    dims = binding.make_dims(x["q"], x["k"], x["profiles"], x["window"], x["query_offset"])
+    ws = binding.alloc_workspace(dims, False, "cuda")
+    assert binding.inkling_rel_attn_validate(dims, x["valid"], x["key_valid"], x["positions"], x["key_positions"],
+                                             ws) == binding.INKLING_OK
+    check_full(x)
