@@ -47,27 +47,42 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
-    h = hashlib.sha256()
+# source files each kernel is built from (its own translation unit and the headers it includes)
+KERNEL_SOURCES = {
+    "fwd:attn_fwd": ["fwd.cu", "common.cuh", "launch.h", "ptx.cuh"],
+    "bwd:attn_bwd_dkdv": ["bwd.cu", "common.cuh", "launch.h", "ptx.cuh"],
+    "bwd:attn_bwd_dq": ["bwd.cu", "common.cuh", "launch.h", "ptx.cuh"],
+    "bwd:bwd_prep": ["prep_kernels.cu", "common.cuh", "launch.h", "ptx.cuh"],
+    "bwd:dprof_zero": ["prep_kernels.cu", "common.cuh", "launch.h", "ptx.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str, read=None) -> str:
+    """sha256 (first 16 hex digits) over the source files of `kernel`. `read(name)` returns a
+    file's bytes (default: the working tree)."""
     csrc = os.path.join(ROOT, "learned_relative_gqa_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+    if read is None:
+        def read(name):
+            with open(os.path.join(csrc, name), "rb") as f:
+                return f.read()
+    h = hashlib.sha256()
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        h.update(name.encode() + read(name))
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it was
-    taken on the current kernel sources; else None."""
+    taken on the current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     k = d.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("bytes_per_launch_full_size")
+    if k is None or k.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return k.get("bytes_per_launch_full_size")
 
 
 class ClockSampler:
