@@ -183,3 +183,83 @@ def allowed_counts(w: Workload, inputs) -> int:
         total += int(cnt.sum())
     del kpos
     return total * w.heads_q
+
+
+# --------------------------------------------------------------------------
+# generic FlexAttention variant (NeMo AutoModel ``FlexAttention`` module page):
+# [B, H, S, D] layout, per-head sink weights, EOS-delimited documents
+# --------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class FlexWorkload:
+    name: str
+    batch: int
+    seq: int
+    heads_q: int
+    heads_kv: int
+    head_dim: int
+    mask_type: str = "causal"                  # "causal" or "block_causal"
+    docs: Optional[Tuple[int, int]] = None     # document length range (block_causal), EOS closes each
+    fixed_block_size: int = 0
+    sliding_window: int = 0
+    sink: bool = True                          # draw sink_weights [Hq]
+    scale: Optional[float] = None
+    eos_id: int = 2
+    vocab: int = 32000
+
+
+FLEX_WORKLOADS = [
+    # the packed-documents shape with EOS-delimited documents, per-head sinks
+    FlexWorkload("flex_packed", 4, 4096, 32, 8, 128, "block_causal", docs=(256, 2048)),
+]
+FLEX_BY_NAME = {w.name: w for w in FLEX_WORKLOADS}
+
+
+def flex_seed_of(w: FlexWorkload) -> int:
+    for idx, x in enumerate(FLEX_WORKLOADS):
+        if x.name == w.name:
+            return 3000 + idx
+    return 4000 + (zlib.crc32(repr(w).encode()) & 0xFFFF)
+
+
+def make_flex_inputs(w: FlexWorkload, device="cpu", seed: Optional[int] = None, with_dout: bool = True):
+    """q [B,Hq,S,D], k / v [B,Hkv,S,D] ~ N(0,1) rounded to BF16, sink_weights [Hq] ~ N(0,1)
+    FP32 (or None), tokens [B,S] int64 and dout [B,Hq,S,D] ~ N(0,1) rounded to BF16.
+
+    Float draws on a generator of the target device (q, k, v, sink_weights, dout in that
+    order); tokens on a CPU generator with the same seed: ids uniform in [0, vocab)
+    without the EOS id, then document lengths ~ U{lo..hi} drawn until they cover the
+    row, the last one truncated, and the EOS id placed on the last token of every
+    complete document.
+    """
+    seed = flex_seed_of(w) if seed is None else seed
+    dev = torch.device(device)
+    g = torch.Generator(dev)
+    g.manual_seed(seed)
+    B, S, Hq, Hkv, D = w.batch, w.seq, w.heads_q, w.heads_kv, w.head_dim
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32)
+
+    q = randn(B, Hq, S, D).to(torch.bfloat16)
+    k = randn(B, Hkv, S, D).to(torch.bfloat16)
+    v = randn(B, Hkv, S, D).to(torch.bfloat16)
+    sink = randn(Hq) if w.sink else None
+    dout = randn(B, Hq, S, D).to(torch.bfloat16) if with_dout else None
+
+    gc = torch.Generator("cpu")
+    gc.manual_seed(seed)
+    tokens = torch.randint(0, w.vocab - 1, (B, S), generator=gc, dtype=torch.int64)
+    tokens = tokens + (tokens >= w.eos_id).to(torch.int64)        # never the EOS id
+    if w.docs is not None:
+        lo, hi = w.docs
+        for b in range(B):
+            c = 0
+            while c < S:
+                L = int(torch.randint(lo, hi + 1, (1,), generator=gc))
+                if c + L <= S:
+                    tokens[b, c + L - 1] = w.eos_id
+                c += L
+    return dict(q=q, k=k, v=v, sink_weights=sink, tokens=tokens.to(dev), dout=dout,
+                mask_type=w.mask_type, eos_id=w.eos_id, fixed_block_size=w.fixed_block_size,
+                sliding_window=w.sliding_window, scale=w.scale, enable_gqa=Hq != Hkv)
+
