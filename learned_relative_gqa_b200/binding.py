@@ -30,6 +30,16 @@ class Dims(ctypes.Structure):
         "batch", "seq_q", "seq_k", "heads_q", "heads_kv", "head_dim", "rel_extent", "window", "query_offset")]
 
 
+class FlexDims(ctypes.Structure):
+    """inkling_flex_attn_dims (include/inkling_flex_attn.h)."""
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "seq", "heads_q", "heads_kv", "head_dim", "mask_type", "fixed_block_size", "sliding_window",
+        "eos_id", "enable_gqa")] + [("scale", ctypes.c_double)]
+
+
+FLEX_MASK_TYPES = {"causal": 0, "block_causal": 1}
+
+
 class InklingError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -70,6 +80,13 @@ def load(path: str = LIB_PATH):
     lib.inkling_rel_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
     lib.inkling_rel_attn_set_timing_events.restype = ctypes.c_int
     lib.inkling_rel_attn_set_timing_events.argtypes = [vp, ctypes.c_int]
+    fd = ctypes.POINTER(FlexDims)
+    lib.inkling_flex_attn_workspace_size.restype = sz
+    lib.inkling_flex_attn_workspace_size.argtypes = [fd, ctypes.c_int]
+    lib.inkling_flex_attn_fwd.restype = ctypes.c_int
+    lib.inkling_flex_attn_fwd.argtypes = [fd] + [vp] * 7 + [vp, sz, vp]
+    lib.inkling_flex_attn_bwd.restype = ctypes.c_int
+    lib.inkling_flex_attn_bwd.argtypes = [fd] + [vp] * 12 + [vp, sz, vp]
     lib.inkling_rel_attn_last_cuda_error.restype = ctypes.c_char_p
     lib.inkling_rel_attn_last_cuda_error.argtypes = []
     lib.inkling_status_string.restype = ctypes.c_char_p
@@ -214,3 +231,73 @@ def backward(q, k, v, profiles, sink, valid, key_valid, positions, key_positions
     inkling_rel_attn_bwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout,
                          dlse, dq, dk, dv, dprof, dsink, ws, stream)
     return dict(dq=dq, dk=dk, dv=dv, dprofiles=dprof, dsink=dsink)
+
+
+# --------------------------------------------------------------------------
+# generic FlexAttention variant (include/inkling_flex_attn.h)
+# --------------------------------------------------------------------------
+def make_flex_dims(q: torch.Tensor, k: torch.Tensor, *, mask_type: str = "causal", eos_id: int = 0,
+                   fixed_block_size: int = 0, sliding_window: int = 0, scale: Optional[float] = None,
+                   enable_gqa: bool = False) -> FlexDims:
+    B, Hq, S, D = q.shape
+    if mask_type not in FLEX_MASK_TYPES:
+        raise ValueError(f"mask_type must be one of {sorted(FLEX_MASK_TYPES)}")
+    return FlexDims(B, S, Hq, k.shape[1], D, FLEX_MASK_TYPES[mask_type], int(fixed_block_size), int(sliding_window),
+                    int(eos_id), int(bool(enable_gqa)), 0.0 if scale is None else float(scale))
+
+
+def inkling_flex_attn_workspace_size(dims: FlexDims, backward: bool) -> int:
+    return int(load().inkling_flex_attn_workspace_size(ctypes.byref(dims), int(bool(backward))))
+
+
+def inkling_flex_attn_fwd(dims: FlexDims, q, k, v, sink_weights, tokens, out, lse, workspace, stream=None) -> None:
+    st = load().inkling_flex_attn_fwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(sink_weights), _p(tokens), _p(out),
+                                      _p(lse), _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_flex_attn_fwd")
+
+
+def inkling_flex_attn_bwd(dims: FlexDims, q, k, v, sink_weights, tokens, out, lse, dout, dq, dk, dv, dsink_weights,
+                          workspace, stream=None) -> None:
+    st = load().inkling_flex_attn_bwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(sink_weights), _p(tokens),
+                                      _p(out), _p(lse), _p(dout), _p(dq), _p(dk), _p(dv), _p(dsink_weights),
+                                      _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_flex_attn_bwd")
+
+
+def _flex_ws(dims: FlexDims, backward: bool, device) -> torch.Tensor:
+    n = inkling_flex_attn_workspace_size(dims, backward)
+    if n == 0:
+        raise InklingError(INKLING_ERR_INVALID_ARG, "inkling_flex_attn_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def flex_forward(q, k, v, sink_weights=None, tokens=None, *, mask_type: str = "causal", eos_id: int = 0,
+                 fixed_block_size: int = 0, sliding_window: int = 0, scale: Optional[float] = None,
+                 enable_gqa: bool = False, workspace=None, stream=None):
+    """out [B,Hq,S,D] BF16 and lse [B,Hq,S] FP32 (see include/inkling_flex_attn.h)."""
+    _contig(q, k, v, sink_weights, tokens)
+    dims = make_flex_dims(q, k, mask_type=mask_type, eos_id=eos_id, fixed_block_size=fixed_block_size,
+                          sliding_window=sliding_window, scale=scale, enable_gqa=enable_gqa)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ws = _flex_ws(dims, False, q.device) if workspace is None else workspace
+    inkling_flex_attn_fwd(dims, q, k, v, sink_weights, tokens, out, lse, ws, stream)
+    return out, lse
+
+
+def flex_backward(q, k, v, out, lse, dout, sink_weights=None, tokens=None, *, mask_type: str = "causal",
+                  eos_id: int = 0, fixed_block_size: int = 0, sliding_window: int = 0,
+                  scale: Optional[float] = None, enable_gqa: bool = False, workspace=None, stream=None):
+    """dict dq [B,Hq,S,D], dk / dv [B,Hkv,S,D] and dsink_weights [Hq] (None without sinks), FP32."""
+    _contig(q, k, v, out, lse, dout, sink_weights, tokens)
+    dims = make_flex_dims(q, k, mask_type=mask_type, eos_id=eos_id, fixed_block_size=fixed_block_size,
+                          sliding_window=sliding_window, scale=scale, enable_gqa=enable_gqa)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(q.shape, **f32)
+    dk = torch.empty(k.shape, **f32)
+    dv = torch.empty(v.shape, **f32)
+    dsw = None if sink_weights is None else torch.empty(sink_weights.shape, **f32)
+    ws = _flex_ws(dims, True, q.device) if workspace is None else workspace
+    inkling_flex_attn_bwd(dims, q, k, v, sink_weights, tokens, out, lse, dout, dq, dk, dv, dsw, ws, stream)
+    return dict(dq=dq, dk=dk, dv=dv, dsink_weights=dsw)
+

@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (ok) {
             const bool row_in = j < p.Skv;
-            float* dst = (w == 0 ? p.dk : p.dv) + ((size_t(b) * p.Skv + j) * p.Hkv + g) * size_t(D);
+            float* dst = (w == 0 ? p.dk : p.dv) + (b * p.kv_sb + j * p.kv_ss + g * p.kv_sh);
             const float mul = (w == 0) ? p.scale : 1.f;
             const uint32_t col = (w == 0) ? L::DK_COL : L::DV_COL;
             if (n_steps > 0) {
@@ -891,7 +891,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
         }
         if (ok) {
-            float* dst = p.dq + ((size_t(b) * p.S + i) * p.Hq + h) * size_t(D);
+            float* dst = p.dq + (b * p.row_sb + i * p.row_ss + h * p.row_sh);
             constexpr int HALF = D / 2;
             if (n_steps > 0) {
 #pragma unroll 1

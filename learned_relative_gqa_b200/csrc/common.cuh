@@ -83,17 +83,24 @@ inline WorkspaceLayout workspace_layout(int64_t B, int64_t S, int64_t Hq, int64_
 // Sizes and pointers shared by the attention kernels.
 struct AttnParams {
     int B, S, Skv, Hq, Hkv, D, R, W, q_off;
-    float scale;          // head_dim^-0.5
+    float scale;          // multiplies q.k (head_dim^-0.5 unless the caller gives another)
     float scale_log2;     // scale * log2(e)
     uint64_t timeout_ns;
     const uint16_t* profiles;
     const void* safe_src;  // any valid 16-B aligned global address (source of zero-fill copies)
-    const float* sink;
+    const float* sink;    // sink of row (b, i, h): sink[b * sink_sb + i * sink_ss + h * sink_sh]
+    int64_t sink_sb, sink_ss, sink_sh;
+    // element strides of the (b, i, h) rows of out and dq, of the (b, i, h) entries of
+    // lse, and of the (b, j, g) rows of dk / dv (the D values of a row are contiguous)
+    int64_t row_sb, row_ss, row_sh;
+    int64_t lse_sb, lse_ss, lse_sh;
+    int64_t kv_sb, kv_ss, kv_sh;
     const int2* row_bounds;
     const TileBounds* tile_bounds;
     int* err;
-    // forward
+    // forward (out_bf16 set: the output is stored as BF16 there, out unused)
     float* out;
+    uint16_t* out_bf16;
     float* lse;
     // backward
     const float* lse2t;

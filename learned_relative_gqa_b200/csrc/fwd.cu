@@ -328,7 +328,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         const bool row_in = i < p.S;
         const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
         const bool empty = rb.x > rb.y;
-        const float sigma = row_in ? p.sink[(size_t(b) * p.S + i) * p.Hq + h] : 0.f;
+        // no sink array: no sink term (a logit of -inf)
+        const float sigma = !row_in ? 0.f : p.sink ? p.sink[b * p.sink_sb + i * p.sink_ss + h * p.sink_sh] : -INFINITY;
         float m2 = sigma * kLog2e;  // running maximum, log2 units
         float l = 1.f;              // running denominator; the sink contributes exp(0)
         bool seen = false;          // some earlier step held an unmasked key of this row
@@ -539,7 +540,19 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         }
         if (ok) {
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            float* orow = p.out + ((size_t(b) * p.S + i) * p.Hq + h) * size_t(D);
+            const int64_t orow_at = b * p.row_sb + i * p.row_ss + h * p.row_sh;
+            float* orow = p.out + orow_at;
+            uint16_t* orow16 = p.out_bf16 ? p.out_bf16 + orow_at : nullptr;
+            auto store4 = [&](int e, float4 v) {  // output columns e .. e + 3
+                if (orow16) {
+                    uint2 u;
+                    u.x = pack_bf16x2(v.x, v.y);
+                    u.y = pack_bf16x2(v.z, v.w);
+                    *reinterpret_cast<uint2*>(orow16 + e) = u;
+                } else {
+                    *reinterpret_cast<float4*>(orow + e) = v;
+                }
+            };
             if (n_steps > 0) {
 #pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -554,17 +567,16 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                             v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * inv_l;
                             v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * inv_l;
                             v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * inv_l;
-                            *reinterpret_cast<float4*>(orow + 32 * c4 + 4 * q) = v;
+                            store4(32 * c4 + 4 * q, v);
                         }
                     }
                 }
             } else if (row_in) {
-                for (int e = 0; e < D; e += 4)
-                    *reinterpret_cast<float4*>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int e = 0; e < D; e += 4) store4(e, make_float4(0.f, 0.f, 0.f, 0.f));
             }
             if (row_in) {
                 const float lse = (empty || n_steps == 0) ? sigma : (m2 + log2f(l)) * kLn2;
-                p.lse[(size_t(b) * p.S + i) * p.Hq + h] = lse;
+                p.lse[b * p.lse_sb + i * p.lse_ss + h * p.lse_sh] = lse;
             }
         }
     }

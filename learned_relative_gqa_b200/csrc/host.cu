@@ -2,13 +2,16 @@
 // include/inkling_rel_attn.h): argument checks, workspace carving, TMA
 // descriptor encoding and the launch sequence of each entry point.
 #include <cstdint>
+#include <cmath>
 #include <cstring>
+#include <functional>
 #include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "inkling_flex_attn.h"
 #include "inkling_rel_attn.h"
 #include "launch.h"
 
@@ -40,13 +43,16 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// BF16 tensor [B, T, H, D] as a 4-D map {D, H, T, B}; box {64, 1, rows, 1};
-// 128-byte swizzle; out-of-range rows read as zero.
-bool encode_bhtd(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t H, int64_t D, int rows) {
+// BF16 tensor [B, T, H, D] (or, with bhsd, [B, H, T, D]) as a 4-D map {D, H, T, B};
+// box {64, 1, rows, 1}; 128-byte swizzle; out-of-range rows read as zero. The kernels
+// address (d, head, row, batch) either way: only the strides differ.
+bool encode_bhtd(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t H, int64_t D, int rows,
+                 bool bhsd = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
-    cuuint64_t strides[3] = {cuuint64_t(D * 2), cuuint64_t(H * D * 2), cuuint64_t(T * H * D * 2)};
+    cuuint64_t strides[3] = {cuuint64_t((bhsd ? T : 1) * D * 2), cuuint64_t((bhsd ? 1 : H) * D * 2),
+                             cuuint64_t(T * H * D * 2)};
     cuuint32_t box[4] = {64u, 1u, cuuint32_t(rows), 1u};
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -211,6 +217,20 @@ AttnParams base_params(const inkling_rel_attn_dims* d, const Ws& w, const uint16
     p.profiles = profiles;
     p.safe_src = w.row_bounds();
     p.sink = sink;
+    // [B, S, H, D] tensors, [B, S, H] sink / lse
+    const int64_t S = d->seq_q, Hq = d->heads_q, D = d->head_dim;
+    p.sink_sb = S * Hq;
+    p.sink_ss = Hq;
+    p.sink_sh = 1;
+    p.row_sb = S * Hq * D;
+    p.row_ss = Hq * D;
+    p.row_sh = D;
+    p.lse_sb = S * Hq;
+    p.lse_ss = Hq;
+    p.lse_sh = 1;
+    p.kv_sb = d->seq_k * d->heads_kv * D;
+    p.kv_ss = d->heads_kv * D;
+    p.kv_sh = D;
     p.row_bounds = w.row_bounds();
     p.tile_bounds = w.tiles();
     p.err = w.ctl();
@@ -255,6 +275,147 @@ inkling_status noalloc_scratch(void** out) {
     }
     *out = g_noalloc_ptr[dev];
     return INKLING_OK;
+}
+
+// Tensor maps of one backward call.
+struct BwdMaps {
+    CUtensorMap tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64, tband;
+};
+
+// The launch sequence of one backward call, for either ABI. `pre_bounds` (optional)
+// runs on the stream of the bounds kernels before them; `prep` launches the backward
+// preprocessing on the stream it is given.
+inkling_status bwd_launches(const inkling_rel_attn_dims* dims, const Ws& w, const AttnParams& p, const BwdMaps& m,
+                            const uint8_t* valid, const uint8_t* key_valid, const int32_t* positions, bool has_keys,
+                            cudaStream_t st, const std::function<cudaError_t(cudaStream_t)>& pre_bounds,
+                            const std::function<cudaError_t(cudaStream_t)>& prep) {
+    LaunchTimer tm(st);
+    // Two streams, except while the timing hook is on (it wants one kernel at a time):
+    //   caller's stream: prep -> (wait row bounds) -> dK/dV
+    //   side stream:     key span, row bounds -> dprofiles zeroing -> (wait prep) -> dQ
+    // dK/dV and dQ read the same inputs and write disjoint outputs; the zeroing writes the
+    // dprofiles entries that dK/dV does not (distances outside a row's visited range).
+    SideStream* side = nullptr;
+    const bool overlap = !tm.active();
+    cudaError_t e = cudaSuccess;
+    if (overlap) {
+        e = side_stream(&side);
+        if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    cudaStream_t st2 = overlap ? side->s : st;
+    auto join = [&](inkling_status r) {  // on the error paths too: no work stays forked off
+        if (overlap) {
+            cudaError_t e2 = cudaEventRecord(side->join, side->s);
+            if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, side->join, 0);
+            if (r == INKLING_OK && e2 != cudaSuccess) r = cuda_status(e2);
+        }
+        return r;
+    };
+    if (pre_bounds) e = pre_bounds(st2);
+    inkling_status s = e == cudaSuccess ? run_bounds(dims, w, valid, key_valid, positions, st2, tm)
+                                        : cuda_status(e);
+    if (s != INKLING_OK) return join(s);
+    if (overlap) e = cudaEventRecord(side->bounds, st2);
+    if (e == cudaSuccess)
+        e = tm.run([&] { return prep(st); });
+    if (e == cudaSuccess && overlap) e = cudaEventRecord(side->ready, st);
+    if (e == cudaSuccess)
+        e = tm.run([&] {
+            return dims->rel_extent > 0 ? launch_dprof_zero(w.row_bounds(), p.B, p.S, p.Hq, p.R, p.q_off,
+                                                            p.dprofiles, st2)
+                                        : cudaSuccess;
+        });
+    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st, side->bounds, 0);
+    if (e == cudaSuccess)
+        e = tm.run([&] { return has_keys ? launch_bwd_dkdv(m.tq64, m.tk128, m.tv128, m.tdo64, m.tband, p, st) : cudaSuccess; });
+    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st2, side->ready, 0);
+    if (e == cudaSuccess) e = tm.run([&] { return launch_bwd_dq(m.tq128, m.tk64, m.tv64, m.tdo128, p, st2); });
+    return join(cuda_status(e));
+}
+
+// ---------------------------------------------------------------------------
+// generic FlexAttention variant
+// ---------------------------------------------------------------------------
+// The learned-relative problem it maps to: no profiles, S queries and S keys, the
+// sliding window as the window, no query offset.
+inkling_status flex_dims(const inkling_flex_attn_dims* f, inkling_rel_attn_dims* d) {
+    if (!f) return INKLING_ERR_INVALID_ARG;
+    if (f->mask_type != INKLING_FLEX_CAUSAL && f->mask_type != INKLING_FLEX_BLOCK_CAUSAL)
+        return INKLING_ERR_INVALID_ARG;
+    if (f->fixed_block_size < 0 || f->sliding_window < 0 || f->heads_q <= 0 || f->heads_kv <= 0)
+        return INKLING_ERR_INVALID_ARG;
+    if (f->heads_q != f->heads_kv && !f->enable_gqa) return INKLING_ERR_INVALID_ARG;
+    if (f->fixed_block_size >= (int64_t(1) << 30)) return INKLING_ERR_UNSUPPORTED;
+    d->batch = f->batch;
+    d->seq_q = f->seq;
+    d->seq_k = f->seq;
+    d->heads_q = f->heads_q;
+    d->heads_kv = f->heads_kv;
+    d->head_dim = f->head_dim;
+    d->rel_extent = 0;
+    d->window = f->sliding_window;
+    d->query_offset = 0;
+    return check_dims(d);
+}
+
+// Workspace: the learned-relative layout, then block positions int32 [B, S], an
+// all-ones validity mask u8 [B, S] and (backward) per-row sink gradients f32 [B, Hq, S].
+struct FlexWs {
+    Ws w;
+    int32_t* positions = nullptr;
+    uint8_t* valid = nullptr;
+    float* dsink_rows = nullptr;
+    size_t total = 0;
+};
+FlexWs flex_layout(const inkling_rel_attn_dims& d, bool backward, uint8_t* base) {
+    FlexWs f;
+    f.w.L = workspace_layout(d.batch, d.seq_q, d.heads_q, d.head_dim, backward);
+    f.w.base = base;
+    size_t off = align_up(f.w.L.total, 256);
+    const size_t pos_off = off;
+    off = align_up(off + size_t(d.batch) * d.seq_q * 4, 256);
+    const size_t valid_off = off;
+    off = align_up(off + size_t(d.batch) * d.seq_q, 256);
+    const size_t dsr_off = off;
+    if (backward) off = align_up(off + size_t(d.batch) * d.heads_q * d.seq_q * 4, 256);
+    f.total = off;
+    if (base) {
+        f.positions = reinterpret_cast<int32_t*>(base + pos_off);
+        f.valid = base + valid_off;
+        f.dsink_rows = backward ? reinterpret_cast<float*>(base + dsr_off) : nullptr;
+    }
+    return f;
+}
+
+// Strides of the [B, H, S, D] tensors, [B, H, S] lse and [Hq] sink weights; the scale.
+void flex_params(AttnParams& p, const inkling_flex_attn_dims* f, const float* sink_weights) {
+    const int64_t S = f->seq, Hq = f->heads_q, Hkv = f->heads_kv, D = f->head_dim;
+    p.scale = (!sink_weights && f->scale > 0) ? float(f->scale) : 1.0f / sqrtf(float(D));
+    p.scale_log2 = p.scale * kLog2e;
+    p.sink = sink_weights;
+    p.sink_sb = 0;
+    p.sink_ss = 0;
+    p.sink_sh = 1;
+    p.row_sb = Hq * S * D;
+    p.row_ss = D;
+    p.row_sh = S * D;
+    p.lse_sb = Hq * S;
+    p.lse_ss = 1;
+    p.lse_sh = S;
+    p.kv_sb = Hkv * S * D;
+    p.kv_ss = D;
+    p.kv_sh = S * D;
+}
+
+// All-ones validity and the block positions, on stream st.
+cudaError_t flex_masks(const inkling_flex_attn_dims* f, const int64_t* tokens, const FlexWs& fw, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(fw.valid, 1, size_t(f->batch) * f->seq, st);
+    if (e == cudaSuccess)
+        e = launch_flex_positions(f->mask_type == INKLING_FLEX_BLOCK_CAUSAL ? tokens : nullptr, f->eos_id,
+                                  int(f->batch), int(f->seq), int(f->fixed_block_size), fw.positions, st);
+    return note(e);
 }
 
 }  // namespace
@@ -400,33 +561,6 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     std::memset(&tband, 0, sizeof(tband));
     if (dims->rel_extent > 0 && !encode_band(&tband, profiles, B * Hq * S, dims->rel_extent)) return INKLING_ERR_CUDA;
 
-    LaunchTimer tm(st);
-    // Two streams, except while the timing hook is on (it wants one kernel at a time):
-    //   caller's stream: prep -> (wait row bounds) -> dK/dV
-    //   side stream:     key span, row bounds -> dprofiles zeroing -> (wait prep) -> dQ
-    // dK/dV and dQ read the same inputs and write disjoint outputs; the zeroing writes the
-    // dprofiles entries that dK/dV does not (distances outside a row's visited range).
-    SideStream* side = nullptr;
-    const bool overlap = !tm.active();
-    cudaError_t e = cudaSuccess;
-    if (overlap) {
-        e = side_stream(&side);
-        if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
-        if (e != cudaSuccess) return cuda_status(e);
-    }
-    cudaStream_t st2 = overlap ? side->s : st;
-    auto join = [&](inkling_status r) {  // on the error paths too: no work stays forked off
-        if (overlap) {
-            cudaError_t e2 = cudaEventRecord(side->join, side->s);
-            if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, side->join, 0);
-            if (r == INKLING_OK && e2 != cudaSuccess) r = cuda_status(e2);
-        }
-        return r;
-    };
-    s = run_bounds(dims, w, valid, key_valid, positions, st2, tm);
-    if (s != INKLING_OK) return join(s);
-    if (overlap) e = cudaEventRecord(side->bounds, st2);
     AttnParams p = base_params(dims, w, profiles, sink);
     p.lse2t = lse2t;
     p.dvt = dvt;
@@ -434,25 +568,12 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
     p.dk = dk;
     p.dv = dv;
     p.dprofiles = dprofiles;
-    if (e == cudaSuccess)
-        e = tm.run([&] {
-            return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq), dsink, dout_bf16,
-                                   lse2t, dvt, st);
-        });
-    if (e == cudaSuccess && overlap) e = cudaEventRecord(side->ready, st);
-    if (e == cudaSuccess)
-        e = tm.run([&] {
-            return dims->rel_extent > 0 ? launch_dprof_zero(w.row_bounds(), int(B), int(S), int(Hq),
-                                                            int(dims->rel_extent), int(dims->query_offset),
-                                                            dprofiles, st2)
-                                        : cudaSuccess;
-        });
-    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st, side->bounds, 0);
-    if (e == cudaSuccess)
-        e = tm.run([&] { return nk > 0 ? launch_bwd_dkdv(tq64, tk128, tv128, tdo64, tband, p, st) : cudaSuccess; });
-    if (e == cudaSuccess && overlap) e = cudaStreamWaitEvent(st2, side->ready, 0);
-    if (e == cudaSuccess) e = tm.run([&] { return launch_bwd_dq(tq128, tk64, tv64, tdo128, p, st2); });
-    return join(cuda_status(e));
+    BwdMaps mp{tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64, tband};
+    return bwd_launches(dims, w, p, mp, valid, key_valid, positions, nk > 0, st, nullptr,
+                        [&](cudaStream_t s0) {
+                            return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq),
+                                                   dsink, dout_bf16, lse2t, dvt, s0);
+                        });
 }
 
 inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
@@ -472,6 +593,97 @@ inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, c
     // device error word itself and rewrites every other scratch byte it reads)
     return inkling_rel_attn_fwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse,
                                 scratch, kNoAllocScratchBytes, stream);
+}
+
+size_t inkling_flex_attn_workspace_size(const inkling_flex_attn_dims* dims, int backward) {
+    inkling_rel_attn_dims d;
+    if (flex_dims(dims, &d) != INKLING_OK) return 0;
+    return flex_layout(d, backward != 0, nullptr).total;
+}
+
+inkling_status inkling_flex_attn_fwd(const inkling_flex_attn_dims* dims, const uint16_t* q, const uint16_t* k,
+                                     const uint16_t* v, const float* sink_weights, const int64_t* tokens,
+                                     uint16_t* out, float* lse, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    inkling_rel_attn_dims d;
+    inkling_status s = flex_dims(dims, &d);
+    if (s != INKLING_OK) return s;
+    const int64_t n = d.batch * d.seq_q;
+    if (n > 0 && (!q || !k || !v || !out || !lse)) return INKLING_ERR_INVALID_ARG;
+    if (n > 0 && dims->mask_type == INKLING_FLEX_BLOCK_CAUSAL && !tokens) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return INKLING_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return INKLING_ERR_INVALID_ARG;
+    FlexWs fw = flex_layout(d, false, static_cast<uint8_t*>(workspace));
+    if (workspace_bytes < fw.total) return INKLING_ERR_INVALID_ARG;
+    if (n == 0) return INKLING_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap tq, tk, tv;
+    if (!encode_bhtd(&tq, q, d.batch, d.seq_q, d.heads_q, d.head_dim, 128, true) ||
+        !encode_bhtd(&tk, k, d.batch, d.seq_k, d.heads_kv, d.head_dim, 64, true) ||
+        !encode_bhtd(&tv, v, d.batch, d.seq_k, d.heads_kv, d.head_dim, 64, true))
+        return INKLING_ERR_CUDA;
+    if (flex_masks(dims, tokens, fw, st) != cudaSuccess) return INKLING_ERR_CUDA;
+    LaunchTimer tm(st);
+    s = run_bounds(&d, fw.w, fw.valid, fw.valid, fw.positions, st, tm);
+    if (s != INKLING_OK) return s;
+    AttnParams p = base_params(&d, fw.w, nullptr, sink_weights);
+    flex_params(p, dims, sink_weights);
+    p.out = nullptr;
+    p.out_bf16 = out;
+    p.lse = lse;
+    return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+}
+
+inkling_status inkling_flex_attn_bwd(const inkling_flex_attn_dims* dims, const uint16_t* q, const uint16_t* k,
+                                     const uint16_t* v, const float* sink_weights, const int64_t* tokens,
+                                     const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
+                                     float* dk, float* dv, float* dsink_weights, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    inkling_rel_attn_dims d;
+    inkling_status s = flex_dims(dims, &d);
+    if (s != INKLING_OK) return s;
+    const int64_t n = d.batch * d.seq_q;
+    if (n > 0 && (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)) return INKLING_ERR_INVALID_ARG;
+    if (n > 0 && dims->mask_type == INKLING_FLEX_BLOCK_CAUSAL && !tokens) return INKLING_ERR_INVALID_ARG;
+    if (sink_weights && !dsink_weights) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return INKLING_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return INKLING_ERR_INVALID_ARG;
+    FlexWs fw = flex_layout(d, true, static_cast<uint8_t*>(workspace));
+    if (workspace_bytes < fw.total) return INKLING_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n == 0)  // no tokens: the sink weights get no gradient
+        return sink_weights ? cuda_status(cudaMemsetAsync(dsink_weights, 0, size_t(d.heads_q) * 4, st)) : INKLING_OK;
+    const int64_t B = d.batch, S = d.seq_q, Hq = d.heads_q, Hkv = d.heads_kv, D = d.head_dim;
+    auto* lse2t = reinterpret_cast<float*>(fw.w.base + fw.w.L.lse2t);
+    auto* dvt = reinterpret_cast<float*>(fw.w.base + fw.w.L.dvt);
+    BwdMaps mp;
+    std::memset(&mp, 0, sizeof(mp));
+    // dO is read by the tensor maps straight from the caller's BF16 [B, H, S, D] tensor
+    if (!encode_bhtd(&mp.tq64, q, B, S, Hq, D, 64, true) || !encode_bhtd(&mp.tq128, q, B, S, Hq, D, 128, true) ||
+        !encode_bhtd(&mp.tdo64, dout, B, S, Hq, D, 64, true) || !encode_bhtd(&mp.tdo128, dout, B, S, Hq, D, 128, true) ||
+        !encode_bhtd(&mp.tk128, k, B, S, Hkv, D, 128, true) || !encode_bhtd(&mp.tv128, v, B, S, Hkv, D, 128, true) ||
+        !encode_bhtd(&mp.tk64, k, B, S, Hkv, D, 64, true) || !encode_bhtd(&mp.tv64, v, B, S, Hkv, D, 64, true))
+        return INKLING_ERR_CUDA;
+    AttnParams p = base_params(&d, fw.w, nullptr, sink_weights);
+    flex_params(p, dims, sink_weights);
+    p.lse2t = lse2t;
+    p.dvt = dvt;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    return bwd_launches(
+        &d, fw.w, p, mp, fw.valid, fw.valid, fw.positions, true, st,
+        [&](cudaStream_t s2) { return flex_masks(dims, tokens, fw, s2); },
+        [&](cudaStream_t s0) {
+            cudaError_t e = launch_flex_bwd_prep(int(D), out, dout, lse, sink_weights, 0, 0, 1, int(B), int(S),
+                                                 int(Hq), fw.dsink_rows, lse2t, dvt, s0);
+            if (e == cudaSuccess && sink_weights)
+                e = launch_flex_dsink_reduce(fw.dsink_rows, int(B), int(S), int(Hq), dsink_weights, s0);
+            return e;
+        });
 }
 
 inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream) {

@@ -21,6 +21,17 @@ cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const flo
 cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
                               cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st);
+
+// Generic FlexAttention variant: block positions from EOS tokens / fixed blocks, the
+// backward preprocessing of BF16 [B, H, S, D] out / dout rows, and the per-head sum of
+// the per-row sink gradients ([B, Hq, S] -> [Hq]).
+cudaError_t launch_flex_positions(const int64_t* tokens, int64_t eos_id, int B, int S, int fbs, int32_t* positions,
+                                  cudaStream_t st);
+cudaError_t launch_flex_bwd_prep(int D, const uint16_t* out, const uint16_t* dout, const float* lse, const float* sink,
+                                 int64_t sink_sb, int64_t sink_ss, int64_t sink_sh, int B, int S, int Hq,
+                                 float* dsink_rows, float* lse2t, float* dvt, cudaStream_t st);
+cudaError_t launch_flex_dsink_reduce(const float* dsink_rows, int B, int S, int Hq, float* dsink_weights,
+                                     cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* t, float* out, int64_t n, cudaStream_t st);
 
 // Forward attention. tm_q: {D, Hq, S, B} box {64,1,128,1}; tm_k / tm_v: {D, Hkv, Skv, B} box {64,1,64,1}.

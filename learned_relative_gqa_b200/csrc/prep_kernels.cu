@@ -254,6 +254,127 @@ __global__ void bwd_prep_kernel(const float* __restrict__ out, const float* __re
     }
 }
 
+// ---------------------------------------------------------------------------
+// generic FlexAttention variant ([B, H, S, D] tensors, BF16 out / dout,
+// per-head sink weights, EOS-delimited documents and fixed blocks)
+// ---------------------------------------------------------------------------
+
+// positions[b, i] = i - (start of the block holding token i), where a block starts at
+// token 0, after every EOS token (block_causal: the EOS closes its document) and, when
+// fixed_block_size F > 0, at every multiple of F. The attention kernels then see one
+// document per block. grid (B), block 1024: each thread takes a contiguous chunk of
+// the row, the block combines the chunks' latest starts with a max-scan.
+__global__ void flex_positions_kernel(const int64_t* __restrict__ tokens, int64_t eos_id, int S, int fbs,
+                                      int32_t* __restrict__ positions) {
+    const int b = blockIdx.x;
+    const int nt = blockDim.x, t = threadIdx.x;
+    const int chunk = (S + nt - 1) / nt;
+    const int c0 = min(S, t * chunk), c1 = min(S, c0 + chunk);
+    const int64_t* row = tokens ? tokens + size_t(b) * S : nullptr;
+    auto starts_block = [&](int c) {
+        return c == 0 || (row && row[c - 1] == eos_id) || (fbs > 0 && c % fbs == 0);
+    };
+    int last = -1;  // latest block start inside this thread's chunk
+    for (int c = c0; c < c1; ++c)
+        if (starts_block(c)) last = c;
+    // inclusive max-scan over the threads (starts only grow with c)
+    __shared__ int warp_last[32];
+    const int lane = t & 31, w = t >> 5;
+    int v = last;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v = max(v, u);
+    }
+    if (lane == 31) warp_last[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        int x = lane < (nt >> 5) ? warp_last[lane] : -1;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x = max(x, u);
+        }
+        warp_last[lane] = x;
+    }
+    __syncthreads();
+    // latest start before this thread's chunk: the scan up to the previous thread
+    int prev = __shfl_up_sync(0xffffffffu, v, 1);
+    if (lane == 0) prev = -1;
+    if (w > 0) prev = max(prev, warp_last[w - 1]);
+    int start = prev;
+    for (int c = c0; c < c1; ++c) {
+        if (starts_block(c)) start = c;
+        positions[size_t(b) * S + c] = c - start;
+    }
+}
+
+// Backward preprocessing of the generic variant: one warp per (b, h, i) row, rows in
+// [B, H, S] order (consecutive rows are consecutive in memory). Reads the BF16 output
+// and output gradient rows, writes Dv = sum_d dO.O, the per-row sink gradient
+// -exp(sigma - lse) Dv and the transposed lse * log2(e) / Dv of the attention kernels.
+template <int D>
+__global__ void flex_bwd_prep_kernel(const uint16_t* __restrict__ out, const uint16_t* __restrict__ dout,
+                                     const float* __restrict__ lse, const float* __restrict__ sink, int64_t sink_sb,
+                                     int64_t sink_ss, int64_t sink_sh, int B, int S, int Hq,
+                                     float* __restrict__ dsink_rows, float* __restrict__ lse2t,
+                                     float* __restrict__ dvt) {
+    constexpr int PER = D / 32;  // BF16 values per lane: 4 (8 bytes) or 2 (4 bytes)
+    const int64_t nrows = int64_t(B) * Hq * S;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t row = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); row < nrows; row += warps) {
+        const uint16_t* o = out + row * D + lane * PER;
+        const uint16_t* g = dout + row * D + lane * PER;
+        float acc = 0.f;
+        if constexpr (PER == 4) {
+            const uint2 a = *reinterpret_cast<const uint2*>(o);
+            const uint2 c = *reinterpret_cast<const uint2*>(g);
+            acc = __uint_as_float(a.x << 16) * __uint_as_float(c.x << 16) +
+                  __uint_as_float(a.x & 0xFFFF0000u) * __uint_as_float(c.x & 0xFFFF0000u) +
+                  __uint_as_float(a.y << 16) * __uint_as_float(c.y << 16) +
+                  __uint_as_float(a.y & 0xFFFF0000u) * __uint_as_float(c.y & 0xFFFF0000u);
+        } else {
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(o);
+            const uint32_t c = *reinterpret_cast<const uint32_t*>(g);
+            acc = __uint_as_float(a << 16) * __uint_as_float(c << 16) +
+                  __uint_as_float(a & 0xFFFF0000u) * __uint_as_float(c & 0xFFFF0000u);
+        }
+        for (int of = 16; of > 0; of >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, of);
+        if (lane == 0) {
+            const int i = int(row % S);
+            const int64_t bh = row / S;
+            const int h = int(bh % Hq), b = int(bh / Hq);
+            const float l = lse[row];
+            const float sg = sink ? sink[b * sink_sb + i * sink_ss + h * sink_sh] : -INFINITY;  // no sink: -inf
+            float ps = 0.f;
+            if (isfinite(l)) ps = expf(sg - l);
+            dsink_rows[row] = -ps * acc;
+            lse2t[row] = l * kLog2e;
+            dvt[row] = acc;
+        }
+    }
+}
+
+// dsink_weights[h] = sum over (b, i) of the per-row sink gradients, in a fixed order
+// (no atomics: the result does not depend on scheduling). grid (Hq), block 256.
+__global__ void flex_dsink_reduce_kernel(const float* __restrict__ dsink_rows, int B, int S, int Hq,
+                                         float* __restrict__ dsink_weights) {
+    const int h = blockIdx.x;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) {
+        const float* r = dsink_rows + (size_t(b) * Hq + h) * S;
+        for (int i = threadIdx.x; i < S; i += blockDim.x) acc += r[i];
+    }
+    __shared__ float part[32];
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float x = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.f;
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (threadIdx.x == 0) dsink_weights[h] = x;
+    }
+}
+
 // Zero the dprofiles entries of each (b, h, i) row that no allowed key
 // reaches: everything outside the visited distances [i_g - hi, i_g - lo].
 // One warp per 32 consecutive rows of one (b, h): lane l reads the bounds of row
@@ -369,6 +490,35 @@ cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int 
     const long long want = (segs + 7) / 8;  // 8 warps per block
     const int blocks = int(want < 148 * 16 ? want : 148 * 16);
     dprof_zero_kernel<<<blocks, 256, 0, st>>>(row_bounds, B, S, Hq, R, q_off, dprof);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_flex_positions(const int64_t* tokens, int64_t eos_id, int B, int S, int fbs, int32_t* positions,
+                                  cudaStream_t st) {
+    if (B == 0 || S == 0) return cudaSuccess;
+    flex_positions_kernel<<<B, 1024, 0, st>>>(tokens, eos_id, S, fbs, positions);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_flex_bwd_prep(int D, const uint16_t* out, const uint16_t* dout, const float* lse, const float* sink,
+                                 int64_t sink_sb, int64_t sink_ss, int64_t sink_sh, int B, int S, int Hq,
+                                 float* dsink_rows, float* lse2t, float* dvt, cudaStream_t st) {
+    const long long rows = (long long)B * S * Hq;
+    if (rows == 0) return cudaSuccess;
+    const int blocks = int(rows / 8 + 1 < 148 * 32 ? rows / 8 + 1 : 148 * 32);
+    if (D == 128)
+        flex_bwd_prep_kernel<128><<<blocks, 256, 0, st>>>(out, dout, lse, sink, sink_sb, sink_ss, sink_sh, B, S, Hq,
+                                                          dsink_rows, lse2t, dvt);
+    else
+        flex_bwd_prep_kernel<64><<<blocks, 256, 0, st>>>(out, dout, lse, sink, sink_sb, sink_ss, sink_sh, B, S, Hq,
+                                                         dsink_rows, lse2t, dvt);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_flex_dsink_reduce(const float* dsink_rows, int B, int S, int Hq, float* dsink_weights,
+                                     cudaStream_t st) {
+    if (Hq == 0) return cudaSuccess;
+    flex_dsink_reduce_kernel<<<Hq, 256, 0, st>>>(dsink_rows, B, S, Hq, dsink_weights);
     return cudaGetLastError();
 }
 

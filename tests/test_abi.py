@@ -1,6 +1,6 @@
 """CPU-only checks of the C-ABI library: it builds, loads, exports every entry
-point declared in include/inkling_rel_attn.h, sizes workspaces, and rejects bad
-arguments on the host before touching the GPU."""
+point declared in include/*.h, sizes workspaces, and rejects bad arguments on
+the host before touching the GPU."""
 import ctypes
 import os
 import re
@@ -8,7 +8,8 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "inkling_rel_attn.h")
+HEADERS = [os.path.join(ROOT, "include", n) for n in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if n.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -19,15 +20,18 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(inkling_\w+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(inkling_\w+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("inkling_rel_attn_fwd", "inkling_rel_attn_bwd", "inkling_rel_attn_validate",
-                 "inkling_rel_attn_workspace_size", "inkling_rel_attn_last_device_error", "inkling_status_string"):
+                 "inkling_rel_attn_workspace_size", "inkling_rel_attn_last_device_error", "inkling_status_string",
+                 "inkling_flex_attn_fwd", "inkling_flex_attn_bwd", "inkling_flex_attn_workspace_size"):
         assert want in names
 
 
@@ -115,3 +119,39 @@ def test_status_strings(lib):
     assert binding.status_string(0) == "ok"
     assert "timed out" in binding.status_string(4)
     assert binding.status_string(77) == "unknown status"
+
+
+def flex_dims(**kw):
+    from learned_relative_gqa_b200.binding import FlexDims
+    base = dict(batch=2, seq=256, heads_q=8, heads_kv=2, head_dim=128, mask_type=1, fixed_block_size=0,
+                sliding_window=0, eos_id=2, enable_gqa=1, scale=0.0)
+    base.update(kw)
+    return FlexDims(**base)
+
+
+def test_flex_workspace_size(lib):
+    from learned_relative_gqa_b200.binding import inkling_flex_attn_workspace_size as ws
+    f, b = ws(flex_dims(), False), ws(flex_dims(), True)
+    assert 0 < f < b
+    assert ws(flex_dims(enable_gqa=0), False) == 0        # Hq != Hkv needs enable_gqa
+    assert ws(flex_dims(heads_q=2, enable_gqa=0), False) > 0
+    assert ws(flex_dims(mask_type=7), False) == 0
+    assert ws(flex_dims(head_dim=80), False) == 0
+    assert ws(flex_dims(sliding_window=-1), False) == 0
+
+
+def test_flex_rejects_bad_arguments_on_host(lib):
+    fake = ctypes.c_void_p(0x10000)
+    d = flex_dims(head_dim=96)
+    assert lib.inkling_flex_attn_fwd(ctypes.byref(d), *([fake] * 7), fake, 1 << 30, None) == 2
+    d = flex_dims()
+    a = [fake] * 7
+    a[4] = None  # block_causal without tokens
+    assert lib.inkling_flex_attn_fwd(ctypes.byref(d), *a, fake, 1 << 30, None) == 1
+    a = [fake] * 7
+    a[0] = ctypes.c_void_p(0x10008)  # misaligned q
+    assert lib.inkling_flex_attn_fwd(ctypes.byref(d), *a, fake, 1 << 30, None) == 1
+    assert lib.inkling_flex_attn_fwd(ctypes.byref(d), *([fake] * 7), fake, 64, None) == 1  # small workspace
+    b = [fake] * 12
+    b[11] = None  # sink weights without a place for their gradient
+    assert lib.inkling_flex_attn_bwd(ctypes.byref(d), *b, fake, 1 << 34, None) == 1
