@@ -8,7 +8,9 @@ dQ) of the ``train`` workload (B2 S8192 Hq32 Hkv4 D128, window 1024, R 1024,
 packed documents; the only workload with a backward). The metric counts only
 allowed (unmasked) score elements E: 4*D*E forward + 10*D*E backward FLOPs.
 The forward of the ``long`` workload (S 32768, R 4096, full causal) is timed
-as well and reported under ``long_fwd``.
+as well and reported under ``long_fwd``, and one forward + backward of the
+generic FlexAttention variant on the packed-documents shape (EOS-delimited
+documents, per-head sinks, [B, H, S, D] tensors) under ``flex_step``.
 
 python bench.py --gpus N --steps K --warmup W [--impl reference]
 Under torchrun each rank runs its own batch (weak scaling, no data-path
@@ -463,6 +465,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0,
                     help="override the workload's sequence length (smaller cases for profiling)")
     ap.add_argument("--long-steps", type=int, default=3, help="forward steps of the long workload (0 = skip)")
+    ap.add_argument("--flex-steps", type=int, default=3,
+                    help="forward + backward steps of the generic FlexAttention variant (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     args = ap.parse_args()
@@ -589,6 +593,11 @@ def main():
         del bl, xl
         torch.cuda.empty_cache()
 
+    # the generic FlexAttention variant (same kernels, [B, H, S, D], BF16 output)
+    flex_step = None
+    if args.flex_steps > 0 and rank == 0:
+        flex_step = flex_run(args.flex_steps, device, peaks)
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         cpu = cpu_baseline(x, D)
@@ -601,12 +610,53 @@ def main():
             "config": run_config(w, x, E, flops_step, world),
             "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
             "roofline": roof, "kernels": kernels, "gpu_launches": gpu_launches,
-            "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks, "long_fwd": long_fwd,
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks, "long_fwd": long_fwd, "flex_step": flex_step,
         }
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def flex_run(steps, device, peaks):
+    """Forward + backward of the generic variant on ``flex_packed`` through its C ABI,
+    preallocated outputs and workspaces; inputs (q, k, v, dout, out: 0.54 GB) exceed L2."""
+    from learned_relative_gqa_b200 import binding, workloads
+    wf = workloads.FLEX_BY_NAME["flex_packed"]
+    xf = workloads.make_flex_inputs(wf, device)
+    E = workloads.flex_allowed_counts(wf, xf)
+    kw = dict(mask_type=wf.mask_type, eos_id=wf.eos_id, fixed_block_size=wf.fixed_block_size,
+              sliding_window=wf.sliding_window, scale=wf.scale, enable_gqa=wf.heads_q != wf.heads_kv)
+    dims = binding.make_flex_dims(xf["q"], xf["k"], **kw)
+    wsf = torch.empty(binding.inkling_flex_attn_workspace_size(dims, False), dtype=torch.uint8, device=device)
+    wsb = torch.empty(binding.inkling_flex_attn_workspace_size(dims, True), dtype=torch.uint8, device=device)
+    out = torch.empty(xf["q"].shape, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(xf["q"].shape[:3], dtype=torch.float32, device=device)
+    f32 = dict(dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty(xf["q"].shape, **f32), torch.empty(xf["k"].shape, **f32), torch.empty(xf["v"].shape, **f32)
+    dsw = torch.empty(xf["sink_weights"].shape, **f32)
+
+    def fwd():
+        binding.inkling_flex_attn_fwd(dims, xf["q"], xf["k"], xf["v"], xf["sink_weights"], xf["tokens"], out, lse, wsf)
+
+    def bwd():
+        binding.inkling_flex_attn_bwd(dims, xf["q"], xf["k"], xf["v"], xf["sink_weights"], xf["tokens"], out, lse,
+                                      xf["dout"], dq, dk, dv, dsw, wsb)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    ms_f = timed(fwd, steps, torch.cuda.synchronize) / steps
+    ms_b = timed(bwd, steps, torch.cuda.synchronize) / steps
+    D = wf.head_dim
+    tf_f = 4.0 * D * E / (ms_f * 1e-3) / 1e12
+    tf_b = 10.0 * D * E / (ms_b * 1e-3) / 1e12
+    tf = 14.0 * D * E / ((ms_f + ms_b) * 1e-3) / 1e12
+    return {"workload": (f"flex_packed: B{wf.batch} S{wf.seq} Hq{wf.heads_q} Hkv{wf.heads_kv} D{D} "
+                         f"{wf.mask_type} docs{wf.docs} sink_weights[Hq], [B,H,S,D], BF16 out"),
+            "allowed_elements": E, "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3),
+            "fwd_tflops": round(tf_f, 1), "bwd_tflops": round(tf_b, 1), "tflops": round(tf, 1),
+            "pct_of_bf16_peak": round(100 * tf / peaks["bf16_tflops"], 1)}
 
 
 def run_config(w, x, E, flops_step, world):

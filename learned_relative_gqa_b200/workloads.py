@@ -263,3 +263,28 @@ def make_flex_inputs(w: FlexWorkload, device="cpu", seed: Optional[int] = None, 
                 mask_type=w.mask_type, eos_id=w.eos_id, fixed_block_size=w.fixed_block_size,
                 sliding_window=w.sliding_window, scale=w.scale, enable_gqa=Hq != Hkv)
 
+
+def flex_allowed_counts(w: FlexWorkload, inputs) -> int:
+    """Number E of allowed (query, key, head) triples of a generic-variant input, for FLOP
+    accounting: per batch row, the blocks (documents closed by EOS, cut further at
+    multiples of fixed_block_size) each contribute the causal pairs inside them, capped
+    by the sliding window."""
+    tokens = inputs["tokens"].cpu()
+    B, S = tokens.shape
+    total = 0
+    for b in range(B):
+        starts = [0]
+        for c in range(1, S):
+            if (w.mask_type == "block_causal" and int(tokens[b, c - 1]) == w.eos_id) or \
+                    (w.fixed_block_size > 0 and c % w.fixed_block_size == 0):
+                starts.append(c)
+        starts.append(S)
+        for a, e in zip(starts[:-1], starts[1:]):
+            L = e - a
+            if w.sliding_window > 0 and w.sliding_window < L:
+                W = w.sliding_window
+                total += W * (W + 1) // 2 + (L - W) * W
+            else:
+                total += L * (L + 1) // 2
+    return total * w.heads_q
+

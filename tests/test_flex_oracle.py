@@ -309,3 +309,12 @@ def test_pins_reject_planted_mistakes(name, monkeypatch):
         except AssertionError:
             failed += 1
     assert failed > 0, f"no pin caught: {name}"
+
+
+@pytest.mark.parametrize("fbs,win,mask", [(0, 0, "block_causal"), (37, 11, "block_causal"), (0, 7, "causal"),
+                                          (16, 0, "causal")])
+def test_flop_count_of_the_generator_matches_the_oracle_mask(fbs, win, mask):
+    w = W.FlexWorkload("count", 2, 300, 4, 2, 8, mask, docs=(5, 60), fixed_block_size=fbs, sliding_window=win)
+    x = W.make_flex_inputs(w)
+    E = sum(int(flex.allowed(w.seq, mask, x["tokens"][b].numpy(), w.eos_id, fbs, win).sum()) for b in range(2))
+    assert W.flex_allowed_counts(w, x) == E * w.heads_q
