@@ -10,7 +10,8 @@ allowed (unmasked) score elements E: 4*D*E forward + 10*D*E backward FLOPs.
 The forward of the ``long`` workload (S 32768, R 4096, full causal) is timed
 as well and reported under ``long_fwd``, and one forward + backward of the
 generic FlexAttention variant on the packed-documents shape (EOS-delimited
-documents, per-head sinks, [B, H, S, D] tensors) under ``flex_step``.
+documents, per-head sinks, [B, H, S, D] tensors) under ``flex_step``, and
+L2Clip forward + backward on q of the training shape under ``l2clip``.
 
 python bench.py --gpus N --steps K --warmup W [--impl reference]
 Under torchrun each rank runs its own batch (weak scaling, no data-path
@@ -467,6 +468,7 @@ def main():
     ap.add_argument("--long-steps", type=int, default=3, help="forward steps of the long workload (0 = skip)")
     ap.add_argument("--flex-steps", type=int, default=3,
                     help="forward + backward steps of the generic FlexAttention variant (0 = skip)")
+    ap.add_argument("--l2clip-steps", type=int, default=5, help="L2Clip forward + backward steps (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     args = ap.parse_args()
@@ -598,6 +600,10 @@ def main():
     if args.flex_steps > 0 and rank == 0:
         flex_step = flex_run(args.flex_steps, device, peaks)
 
+    l2c = None
+    if args.l2clip_steps > 0 and rank == 0:
+        l2c = l2clip_run(args.l2clip_steps, device, peaks)
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         cpu = cpu_baseline(x, D)
@@ -611,6 +617,7 @@ def main():
             "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
             "roofline": roof, "kernels": kernels, "gpu_launches": gpu_launches,
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks, "long_fwd": long_fwd, "flex_step": flex_step,
+            "l2clip": l2c,
         }
         print(json.dumps(line))
     if dist is not None:
@@ -657,6 +664,45 @@ def flex_run(steps, device, peaks):
             "allowed_elements": E, "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3),
             "fwd_tflops": round(tf_f, 1), "bwd_tflops": round(tf_b, 1), "tflops": round(tf, 1),
             "pct_of_bf16_peak": round(100 * tf / peaks["bf16_tflops"], 1)}
+
+
+def l2clip_run(steps, device, peaks):
+    """L2Clip forward and backward (learned scales and length scaling on) on q of the
+    training shape, B2 S8192 Hq32 D128: 134 MB of BF16 x; both passes are HBM streams
+    (4 and 10 bytes per element), each larger than L2."""
+    from learned_relative_gqa_b200 import binding
+    B, S, H, D = 2, 8192, 32, 128
+    g = torch.Generator(device)
+    g.manual_seed(7)
+    x = torch.randn(B, S, H, D, generator=g, device=device).to(torch.bfloat16)
+    scale = 0.5 + torch.rand(H, D, generator=g, device=device)
+    tau = 0.5 + torch.rand(B, S, generator=g, device=device)
+    dy = torch.randn(B, S, H, D, generator=g, device=device)
+    dims = binding.make_l2clip_dims(x, 9.0)
+    y = torch.empty_like(x)
+    dx = torch.empty(x.shape, dtype=torch.float32, device=device)
+    dscale = torch.empty(H, D, dtype=torch.float32, device=device)
+    dtau = torch.empty(B, S, dtype=torch.float32, device=device)
+    ws = torch.empty(binding.inkling_l2clip_workspace_size(dims), dtype=torch.uint8, device=device)
+
+    def fwd():
+        binding.inkling_l2clip_fwd(dims, x, scale, tau, y)
+
+    def bwd():
+        binding.inkling_l2clip_bwd(dims, x, scale, tau, dy, dx, dscale, dtau, ws)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    ms_f = timed(fwd, steps, torch.cuda.synchronize) / steps
+    ms_b = timed(bwd, steps, torch.cuda.synchronize) / steps
+    n = B * S * H * D
+    bf, bb = 4.0 * n, 10.0 * n
+    return {"workload": f"L2Clip on q: B{B} S{S} H{H} D{D}, learned scales, tau, threshold 9",
+            "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+            "fwd_gbs": round(bf / (ms_f * 1e-3) / 1e9, 1), "bwd_gbs": round(bb / (ms_b * 1e-3) / 1e9, 1),
+            "fwd_frac_of_hbm": round(bf / (ms_f * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+            "bwd_frac_of_hbm": round(bb / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
 
 
 def run_config(w, x, E, flops_step, world):

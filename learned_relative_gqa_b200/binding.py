@@ -40,6 +40,11 @@ class FlexDims(ctypes.Structure):
 FLEX_MASK_TYPES = {"causal": 0, "block_causal": 1}
 
 
+class L2ClipDims(ctypes.Structure):
+    """inkling_l2clip_dims (include/inkling_l2clip.h)."""
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seq", "heads", "head_dim")] + [("threshold", ctypes.c_double)]
+
+
 class InklingError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -87,6 +92,13 @@ def load(path: str = LIB_PATH):
     lib.inkling_flex_attn_fwd.argtypes = [fd] + [vp] * 7 + [vp, sz, vp]
     lib.inkling_flex_attn_bwd.restype = ctypes.c_int
     lib.inkling_flex_attn_bwd.argtypes = [fd] + [vp] * 12 + [vp, sz, vp]
+    ld = ctypes.POINTER(L2ClipDims)
+    lib.inkling_l2clip_workspace_size.restype = sz
+    lib.inkling_l2clip_workspace_size.argtypes = [ld]
+    lib.inkling_l2clip_fwd.restype = ctypes.c_int
+    lib.inkling_l2clip_fwd.argtypes = [ld] + [vp] * 4 + [vp]
+    lib.inkling_l2clip_bwd.restype = ctypes.c_int
+    lib.inkling_l2clip_bwd.argtypes = [ld] + [vp] * 7 + [vp, sz, vp]
     lib.inkling_rel_attn_last_cuda_error.restype = ctypes.c_char_p
     lib.inkling_rel_attn_last_cuda_error.argtypes = []
     lib.inkling_status_string.restype = ctypes.c_char_p
@@ -300,4 +312,52 @@ def flex_backward(q, k, v, out, lse, dout, sink_weights=None, tokens=None, *, ma
     ws = _flex_ws(dims, True, q.device) if workspace is None else workspace
     inkling_flex_attn_bwd(dims, q, k, v, sink_weights, tokens, out, lse, dout, dq, dk, dv, dsw, ws, stream)
     return dict(dq=dq, dk=dk, dv=dv, dsink_weights=dsw)
+
+
+# --------------------------------------------------------------------------
+# L2Clip (include/inkling_l2clip.h)
+# --------------------------------------------------------------------------
+def make_l2clip_dims(x: torch.Tensor, threshold: float) -> L2ClipDims:
+    B, S, H, D = x.shape
+    return L2ClipDims(B, S, H, D, float(threshold))
+
+
+def inkling_l2clip_workspace_size(dims: L2ClipDims) -> int:
+    return int(load().inkling_l2clip_workspace_size(ctypes.byref(dims)))
+
+
+def inkling_l2clip_fwd(dims: L2ClipDims, x, scale, tau, y, stream=None) -> None:
+    _check(load().inkling_l2clip_fwd(ctypes.byref(dims), _p(x), _p(scale), _p(tau), _p(y), _stream(stream)),
+           "inkling_l2clip_fwd")
+
+
+def inkling_l2clip_bwd(dims: L2ClipDims, x, scale, tau, dy, dx, dscale, dtau, workspace, stream=None) -> None:
+    _check(load().inkling_l2clip_bwd(ctypes.byref(dims), _p(x), _p(scale), _p(tau), _p(dy), _p(dx), _p(dscale),
+                                     _p(dtau), _p(workspace), workspace.numel(), _stream(stream)),
+           "inkling_l2clip_bwd")
+
+
+def l2clip_forward(x, threshold: float, scale=None, tau=None, stream=None):
+    """y [B,S,H,D] BF16: x (BF16) clipped per head vector (see include/inkling_l2clip.h)."""
+    _contig(x, scale, tau)
+    dims = make_l2clip_dims(x, threshold)
+    y = torch.empty_like(x)
+    inkling_l2clip_fwd(dims, x, scale, tau, y, stream)
+    return y
+
+
+def l2clip_backward(x, dy, threshold: float, scale=None, tau=None, stream=None):
+    """dict dx [B,S,H,D], dscale [H,D] (None without scale), dtau [B,S] (None without tau), FP32."""
+    _contig(x, dy, scale, tau)
+    dims = make_l2clip_dims(x, threshold)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    dx = torch.empty(x.shape, **f32)
+    dscale = None if scale is None else torch.empty(scale.shape, **f32)
+    dtau = None if tau is None else torch.empty(tau.shape, **f32)
+    n = inkling_l2clip_workspace_size(dims)
+    if n == 0:
+        raise InklingError(INKLING_ERR_INVALID_ARG, "inkling_l2clip_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+    inkling_l2clip_bwd(dims, x, scale, tau, dy, dx, dscale, dtau, ws, stream)
+    return dict(dx=dx, dscale=dscale, dtau=dtau)
 

@@ -155,3 +155,22 @@ def test_flex_rejects_bad_arguments_on_host(lib):
     b = [fake] * 12
     b[11] = None  # sink weights without a place for their gradient
     assert lib.inkling_flex_attn_bwd(ctypes.byref(d), *b, fake, 1 << 34, None) == 1
+
+
+def test_l2clip_rejects_bad_arguments_on_host(lib):
+    from learned_relative_gqa_b200.binding import L2ClipDims
+    fake = ctypes.c_void_p(0x10000)
+    good = L2ClipDims(2, 64, 8, 128, 1.0)
+    assert lib.inkling_l2clip_workspace_size(ctypes.byref(good)) > 0
+    assert lib.inkling_l2clip_workspace_size(ctypes.byref(L2ClipDims(2, 64, 8, 96, 1.0))) == 0
+    assert lib.inkling_l2clip_fwd(ctypes.byref(L2ClipDims(2, 64, 8, 128, -1.0)), fake, None, None, fake, None) == 1
+    assert lib.inkling_l2clip_fwd(ctypes.byref(L2ClipDims(2, 64, 8, 128, float("nan"))), fake, None, None, fake,
+                                  None) == 1
+    assert lib.inkling_l2clip_fwd(ctypes.byref(good), None, None, None, fake, None) == 1
+    assert lib.inkling_l2clip_fwd(ctypes.byref(good), ctypes.c_void_p(0x10004), None, None, fake, None) == 1
+    # a learned scale needs a place for its gradient, and the reverse
+    assert lib.inkling_l2clip_bwd(ctypes.byref(good), fake, fake, None, fake, fake, None, None, fake, 1 << 30,
+                                  None) == 1
+    assert lib.inkling_l2clip_bwd(ctypes.byref(good), fake, None, None, fake, fake, None, fake, fake, 1 << 30,
+                                  None) == 1
+    assert lib.inkling_l2clip_bwd(ctypes.byref(good), fake, None, None, fake, fake, None, None, fake, 16, None) == 1
