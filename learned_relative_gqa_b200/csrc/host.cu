@@ -113,23 +113,33 @@ struct LaunchTimer {
     bool active() const { return g_events != nullptr; }
 };
 
-// Per host thread and device: a second stream and two events, so that the dK/dV and
+// Per host thread and device: a second stream and its events, so that the dK/dV and
 // dQ kernels of one backward call can run side by side (each fills the other's last,
 // partial wave of CTAs). Fork: the side stream waits for the caller's stream; join:
-// the caller's stream waits for the side stream. Works under stream capture.
+// the caller's stream waits for the side stream; both are events, so a stream capture
+// of the caller's stream takes the side stream's work into the graph. The stream is
+// created on the first use outside a capture; a first use inside one gets *out = nullptr
+// (the call then runs on the caller's stream alone).
 struct SideStream {
     int device = -1;
     cudaStream_t s = nullptr;
     cudaEvent_t fork = nullptr, bounds = nullptr, ready = nullptr, join = nullptr;
 };
-cudaError_t side_stream(SideStream** out) {
+cudaError_t side_stream(SideStream** out, cudaStream_t caller) {
     thread_local SideStream per_dev[16];
+    *out = nullptr;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
     SideStream& r = per_dev[dev];
     if (r.s == nullptr) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(caller, &cs) != cudaSuccess) {
+            (void)cudaGetLastError();  // not sticky; leave no error behind for the launches
+            cs = cudaStreamCaptureStatusActive;
+        }
+        if (cs != cudaStreamCaptureStatusNone) return cudaSuccess;
         e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.bounds, cudaEventDisableTiming);
@@ -296,11 +306,15 @@ inkling_status bwd_launches(const inkling_rel_attn_dims* dims, const Ws& w, cons
     // dK/dV and dQ read the same inputs and write disjoint outputs; the zeroing writes the
     // dprofiles entries that dK/dV does not (distances outside a row's visited range).
     SideStream* side = nullptr;
-    const bool overlap = !tm.active();
+    bool overlap = !tm.active();
     cudaError_t e = cudaSuccess;
     if (overlap) {
-        e = side_stream(&side);
-        if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
+        e = side_stream(&side, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        overlap = side != nullptr;
+    }
+    if (overlap) {
+        e = cudaEventRecord(side->fork, st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
         if (e != cudaSuccess) return cuda_status(e);
     }
