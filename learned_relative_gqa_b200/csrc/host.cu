@@ -434,6 +434,12 @@ cudaError_t flex_masks(const inkling_flex_attn_dims* f, const int64_t* tokens, c
 
 }  // namespace
 
+namespace ira {
+// Lets the other translation units' entry points record their CUDA errors for
+// inkling_rel_attn_last_cuda_error.
+cudaError_t note_cuda_error(cudaError_t e) { return note(e); }
+}  // namespace ira
+
 extern "C" {
 
 size_t inkling_rel_attn_workspace_size(const inkling_rel_attn_dims* dims, int backward) {

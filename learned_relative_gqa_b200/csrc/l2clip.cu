@@ -19,6 +19,10 @@
 
 #include "inkling_l2clip.h"
 
+namespace ira {
+cudaError_t note_cuda_error(cudaError_t e);  // host.cu: keeps the error for inkling_rel_attn_last_cuda_error
+}
+
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
@@ -249,7 +253,7 @@ inkling_status check(const inkling_l2clip_dims* d) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inkling_status status_of(cudaError_t e) { return e == cudaSuccess ? INKLING_OK : INKLING_ERR_CUDA; }
+inkling_status status_of(cudaError_t e) { return ira::note_cuda_error(e) == cudaSuccess ? INKLING_OK : INKLING_ERR_CUDA; }
 
 }  // namespace
 
