@@ -192,6 +192,13 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_threads() -> int:
+    """Give the oracle every core this process may use (a launcher such as torchrun sets
+    OMP_NUM_THREADS=1 per rank) and return the thread count it then runs with."""
+    import oracle
+    return oracle.set_threads(cpu_cores())
+
+
 # ---------------------------------------------------------------------------
 # oracle sample (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
@@ -255,6 +262,7 @@ def calibrate_sample(x, target_s: float = 8.0, max_s: float = 20.0):
 
 
 def cpu_baseline(x, D, budget_s=20.0):
+    threads = oracle_threads()
     s_sub, hc, E, dt = calibrate_sample(x, max_s=budget_s)
     if dt < 5.0:  # re-time on the chosen sample
         reps = max(1, int(5.0 / max(dt, 1e-3)))
@@ -264,7 +272,7 @@ def cpu_baseline(x, D, budget_s=20.0):
         dt = (time.perf_counter() - t0) / reps
     flops = 14.0 * D * E
     G = hc["q"].shape[2]
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": (f"FP64 oracle forward+backward on batch 0, one KV group ({G} query heads), first {s_sub} "
                        f"tokens of the same workload: E={E} allowed elements, {dt:.2f} s per step")}
 
@@ -721,6 +729,7 @@ def run_reference(args, w, backward):
     x = workloads.make_inputs(w, "cpu")
     D = w.head_dim
     E_full = workloads.allowed_counts(w, x)
+    threads = oracle_threads()
     s_sub, hc, E, dt = calibrate_sample(x, target_s=4.0, max_s=15.0)
     for _ in range(min(args.warmup, 1)):
         oracle_sample_step(hc)
@@ -737,7 +746,7 @@ def run_reference(args, w, backward):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": run_config(w, x, E_full, (14.0 if backward else 4.0) * D * E_full, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))

@@ -57,6 +57,10 @@ def _bind(lib):
     lib.oracle_bwd_sampled_f64.restype = ctypes.c_int
     lib.oracle_bwd_sampled_f64.argtypes = ([ctypes.POINTER(_Dims)] + [vp] * 11
                                            + [vp, ctypes.c_int64, vp, ctypes.c_int64] + [vp] * 5)
+    lib.oracle_set_threads.restype = None
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.oracle_threads.restype = ctypes.c_int
+    lib.oracle_threads.argtypes = []
     lib.oracle_decode_bf16.restype = None
     lib.oracle_decode_bf16.argtypes = [vp, vp, ctypes.c_int64]
     return lib
@@ -82,6 +86,13 @@ def _ptr(a: Optional[np.ndarray]):
 
 def _f64(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def set_threads(n: int) -> int:
+    """Use n OpenMP threads in the oracle's parallel loops; returns the count now in effect."""
+    lib = load()
+    lib.oracle_set_threads(int(n))
+    return int(lib.oracle_threads())
 
 
 def decode_bf16(bits: np.ndarray) -> np.ndarray:

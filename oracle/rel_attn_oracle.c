@@ -48,6 +48,7 @@
  * exactly by a bit shift. OpenMP parallelises over independent rows.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -75,6 +76,12 @@ static double bf16_bits_to_double(uint16_t bits) {
     memcpy(&f, &u, sizeof f);
     return (double)f;
 }
+
+/* OpenMP threads of the parallel loops below: set (n > 0) and query. */
+void oracle_set_threads(int n) {
+    if (n > 0) omp_set_num_threads(n);
+}
+int oracle_threads(void) { return omp_get_max_threads(); }
 
 void oracle_decode_bf16(const uint16_t* src, double* dst, int64_t n) {
     for (int64_t t = 0; t < n; ++t) dst[t] = bf16_bits_to_double(src[t]);
