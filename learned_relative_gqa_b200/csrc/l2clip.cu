@@ -198,23 +198,39 @@ __global__ void l2clip_bwd_kernel(const uint16_t* __restrict__ x, const float* _
 }
 
 // dtau[t] = sum over h of the parts (threads [0, T)); dscale[j] = sum over chunks of
-// the parts (threads [T, T + H * D)); fixed summation order.
+// the parts (threads [T, T + H * D)); fixed summation order, four partial sums per
+// thread so that four loads are in flight.
 __global__ void l2clip_reduce_kernel(const float* __restrict__ dtau_part, int64_t T, int H,
                                      float* __restrict__ dtau, const float* __restrict__ dscale_part,
                                      int64_t nchunks, int64_t HD, float* __restrict__ dscale) {
     const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i < T) {
         if (dtau) {
-            float a = 0.f;
-            for (int h = 0; h < H; ++h) a += dtau_part[i * H + h];
-            dtau[i] = a;
+            const float* q = dtau_part + i * H;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            int h = 0;
+            for (; h + 3 < H; h += 4) {
+                a0 += q[h];
+                a1 += q[h + 1];
+                a2 += q[h + 2];
+                a3 += q[h + 3];
+            }
+            for (; h < H; ++h) a0 += q[h];
+            dtau[i] = (a0 + a1) + (a2 + a3);
         }
     } else if (i - T < HD) {
         if (dscale) {
-            const int64_t j = i - T;
-            float a = 0.f;
-            for (int64_t c = 0; c < nchunks; ++c) a += dscale_part[c * HD + j];
-            dscale[j] = a;
+            const float* q = dscale_part + (i - T);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            int64_t c = 0;
+            for (; c + 3 < nchunks; c += 4) {
+                a0 += q[c * HD];
+                a1 += q[(c + 1) * HD];
+                a2 += q[(c + 2) * HD];
+                a3 += q[(c + 3) * HD];
+            }
+            for (; c < nchunks; ++c) a0 += q[c * HD];
+            dscale[i - T] = (a0 + a1) + (a2 + a3);
         }
     }
 }

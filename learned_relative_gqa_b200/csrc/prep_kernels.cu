@@ -355,15 +355,25 @@ __global__ void flex_bwd_prep_kernel(const uint16_t* __restrict__ out, const uin
 }
 
 // dsink_weights[h] = sum over (b, i) of the per-row sink gradients, in a fixed order
-// (no atomics: the result does not depend on scheduling). grid (Hq), block 256.
+// (no atomics: the result does not depend on scheduling). grid (Hq), block 1024; each
+// thread keeps four partial sums so that four loads are in flight.
 __global__ void flex_dsink_reduce_kernel(const float* __restrict__ dsink_rows, int B, int S, int Hq,
                                          float* __restrict__ dsink_weights) {
     const int h = blockIdx.x;
-    float acc = 0.f;
+    const int nt = blockDim.x;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int b = 0; b < B; ++b) {
         const float* r = dsink_rows + (size_t(b) * Hq + h) * S;
-        for (int i = threadIdx.x; i < S; i += blockDim.x) acc += r[i];
+        int i = threadIdx.x;
+        for (; i + 3 * nt < S; i += 4 * nt) {
+            a0 += r[i];
+            a1 += r[i + nt];
+            a2 += r[i + 2 * nt];
+            a3 += r[i + 3 * nt];
+        }
+        for (; i < S; i += nt) a0 += r[i];
     }
+    float acc = (a0 + a1) + (a2 + a3);
     __shared__ float part[32];
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
@@ -518,7 +528,7 @@ cudaError_t launch_flex_bwd_prep(int D, const uint16_t* out, const uint16_t* dou
 cudaError_t launch_flex_dsink_reduce(const float* dsink_rows, int B, int S, int Hq, float* dsink_weights,
                                      cudaStream_t st) {
     if (Hq == 0) return cudaSuccess;
-    flex_dsink_reduce_kernel<<<Hq, 256, 0, st>>>(dsink_rows, B, S, Hq, dsink_weights);
+    flex_dsink_reduce_kernel<<<Hq, 1024, 0, st>>>(dsink_rows, B, S, Hq, dsink_weights);
     return cudaGetLastError();
 }
 
