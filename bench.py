@@ -151,6 +151,7 @@ class ClockSampler:
                 self.sample()  # the state right at the end of the timed region
             except Exception:
                 pass
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             with open(self.path, "w") as f:
                 f.write("time,sm_mhz,sm_max_mhz,power_w,reasons_mask\n")
                 for r in self.rows:
@@ -478,6 +479,8 @@ def main():
                     help="forward + backward steps of the generic FlexAttention variant (0 = skip)")
     ap.add_argument("--l2clip-steps", type=int, default=5, help="L2Clip forward + backward steps (0 = skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-csv-dir", default="/tmp",
+                    help="directory for the CSV of the SM clock samples taken during the timed regions")
     ap.add_argument("--e2e-steps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -529,8 +532,7 @@ def main():
     for _ in range(args.warmup):
         step()
     sync_all()
-    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, f"/tmp/clocks_rank{rank}.csv")
+    sampler = ClockSampler(local, os.path.join(args.clock_csv_dir, f"clocks_rank{rank}.csv"))
     ms = timed(step, args.steps, sync_all)
     clocks = sampler.stop()
     ms_t = torch.tensor([ms], device=device, dtype=torch.float64)
@@ -592,8 +594,7 @@ def main():
         for _ in range(2):
             bl.fwd()
         torch.cuda.synchronize()
-        sampler_l = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_long_rank{rank}.csv")) \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, f"/tmp/clocks_long_rank{rank}.csv")
+        sampler_l = ClockSampler(local, os.path.join(args.clock_csv_dir, f"clocks_long_rank{rank}.csv"))
         ms_l = timed(bl.fwd, args.long_steps, torch.cuda.synchronize) / args.long_steps
         clocks_l = sampler_l.stop()
         tfl = 4.0 * wl.head_dim * El / (ms_l * 1e-3) / 1e12
