@@ -99,6 +99,7 @@ class ClockSampler:
     def __init__(self, device_index: int, path: str, period_s: float = 0.004):
         import threading
         self.path, self.period = path, period_s
+        os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
         self.rows, self.proc, self.thread = [], None, None
         self.stop_evt = threading.Event()
         try:
@@ -151,7 +152,6 @@ class ClockSampler:
                 self.sample()  # the state right at the end of the timed region
             except Exception:
                 pass
-            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             with open(self.path, "w") as f:
                 f.write("time,sm_mhz,sm_max_mhz,power_w,reasons_mask\n")
                 for r in self.rows:
