@@ -385,9 +385,18 @@ struct FlexWs {
 };
 FlexWs flex_layout(const inkling_rel_attn_dims& d, bool backward, uint8_t* base) {
     FlexWs f;
-    f.w.L = workspace_layout(d.batch, d.seq_q, d.heads_q, d.head_dim, backward);
+    // the forward sections, then (backward) lse * log2(e) and Dv: the kernels read dO
+    // straight from the caller's BF16 tensor, so there is no BF16 copy of it
+    f.w.L = workspace_layout(d.batch, d.seq_q, d.heads_q, d.head_dim, false);
     f.w.base = base;
     size_t off = align_up(f.w.L.total, 256);
+    if (backward) {
+        const size_t rows = size_t(d.batch) * d.heads_q * d.seq_q;
+        f.w.L.lse2t = off;
+        off = align_up(off + rows * 4, 256);
+        f.w.L.dvt = off;
+        off = align_up(off + rows * 4, 256);
+    }
     const size_t pos_off = off;
     off = align_up(off + size_t(d.batch) * d.seq_q * 4, 256);
     const size_t valid_off = off;
