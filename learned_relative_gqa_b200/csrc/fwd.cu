@@ -554,22 +554,43 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 }
             };
             if (n_steps > 0) {
+                // 32 x 32 chunks go out through this warp's own 32 band rows (idle now: every
+                // copy into them has completed), 144-byte pitch: each lane writes its row,
+                // then 8 lanes store 128 contiguous bytes of one row, four rows per store
+                float* const stage = reinterpret_cast<float*>(band0 + 32 * wq * BAND_PITCH);
+                constexpr int SP = BAND_PITCH / 4;  // staging row pitch in floats
+                const int sr = lane >> 3, sc = 4 * (lane & 7);
 #pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + L::o_col(s) + 32 * c4, o);
                     tmem_wait_ld();
-                    if (row_in) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 v;
-                            v.x = empty ? 0.f : __uint_as_float(o[4 * q + 0]) * inv_l;
-                            v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * inv_l;
-                            v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * inv_l;
-                            v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * inv_l;
-                            store4(32 * c4 + 4 * q, v);
+                    for (int q = 0; q < 8; ++q) {
+                        float4 v;
+                        v.x = empty ? 0.f : __uint_as_float(o[4 * q + 0]) * inv_l;
+                        v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * inv_l;
+                        v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * inv_l;
+                        v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * inv_l;
+                        *reinterpret_cast<float4*>(stage + lane * SP + 4 * q) = v;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + sr;           // row of this warp
+                        const int ir = i0 + 32 * wq + rr;    // its query row
+                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * SP + sc);
+                        if (ir < p.S) {
+                            const int64_t at = b * p.row_sb + ir * p.row_ss + h * p.row_sh + 32 * c4 + sc;
+                            if (p.out_bf16) {
+                                *reinterpret_cast<uint2*>(p.out_bf16 + at) =
+                                    make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                            } else {
+                                *reinterpret_cast<float4*>(p.out + at) = v;
+                            }
                         }
                     }
+                    __syncwarp();
                 }
             } else if (row_in) {
                 for (int e = 0; e < D; e += 4) store4(e, make_float4(0.f, 0.f, 0.f, 0.f));
