@@ -477,23 +477,35 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) {
             const bool row_in = j < p.Skv;
             float* dst = (w == 0 ? p.dk : p.dv) + (b * p.kv_sb + j * p.kv_ss + g * p.kv_sh);
+            float* const base = (w == 0 ? p.dk : p.dv) + (b * p.kv_sb + g * p.kv_sh);
             const float mul = (w == 0) ? p.scale : 1.f;
             const uint32_t col = (w == 0) ? L::DK_COL : L::DV_COL;
             if (n_steps > 0) {
+                // 32 x 32 chunks go out through shared memory (the key / query tiles, idle once
+                // every MMA has completed), 144-byte pitch per row: each lane writes its row,
+                // then 8 lanes store 128 contiguous bytes of one row, four rows per store
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * 36;
+                const int sr = lane >> 3, sc = 4 * (lane & 7);
 #pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + col + 32 * c4, o);
                     tmem_wait_ld();
-                    if (row_in) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 v = make_float4(__uint_as_float(o[4 * q]) * mul, __uint_as_float(o[4 * q + 1]) * mul,
-                                                   __uint_as_float(o[4 * q + 2]) * mul,
-                                                   __uint_as_float(o[4 * q + 3]) * mul);
-                            *reinterpret_cast<float4*>(dst + 32 * c4 + 4 * q) = v;
-                        }
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4*>(stage + lane * 36 + 4 * q) =
+                            make_float4(__uint_as_float(o[4 * q]) * mul, __uint_as_float(o[4 * q + 1]) * mul,
+                                        __uint_as_float(o[4 * q + 2]) * mul, __uint_as_float(o[4 * q + 3]) * mul);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + sr;          // row of this warp
+                        const int jr = j0 + 32 * wq + rr;   // its key
+                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * 36 + sc);
+                        if (jr < p.Skv) *reinterpret_cast<float4*>(base + jr * p.kv_ss + 32 * c4 + sc) = v;
                     }
+                    __syncwarp();
                 }
             } else if (row_in) {
                 for (int e = 0; e < D; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -892,25 +904,39 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (ok) {
             float* dst = p.dq + (b * p.row_sb + i * p.row_ss + h * p.row_sh);
+            float* const base = p.dq + (b * p.row_sb + h * p.row_sh);
             constexpr int HALF = D / 2;
             if (n_steps > 0) {
+                // 32 x 32 chunks go out through shared memory (the K / V rings, idle once every
+                // MMA has completed), 144-byte pitch per row: each lane writes its row, then
+                // 8 lanes store 128 contiguous bytes of one row, four rows per store
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * 36;
+                const int sr = lane >> 3, sc = 4 * (lane & 7);
 #pragma unroll 1
                 for (int c4 = 0; c4 < HALF / 32; ++c4) {
                     const int col = w * HALF + 32 * c4;
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + L::DQ_COL + col, o);
                     tmem_wait_ld();
-                    if (row_in) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 v;
-                            v.x = empty ? 0.f : __uint_as_float(o[4 * q]) * p.scale;
-                            v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * p.scale;
-                            v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * p.scale;
-                            v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * p.scale;
-                            *reinterpret_cast<float4*>(dst + col + 4 * q) = v;
-                        }
+                    for (int q = 0; q < 8; ++q) {
+                        float4 v;
+                        v.x = empty ? 0.f : __uint_as_float(o[4 * q]) * p.scale;
+                        v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * p.scale;
+                        v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * p.scale;
+                        v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * p.scale;
+                        *reinterpret_cast<float4*>(stage + lane * 36 + 4 * q) = v;
                     }
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + sr;          // row of this warp
+                        const int ir = i0 + 32 * wq + rr;   // its query row
+                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * 36 + sc);
+                        if (ir < p.S) *reinterpret_cast<float4*>(base + ir * p.row_ss + col + sc) = v;
+                    }
+                    __syncwarp();
                 }
             } else if (row_in) {
                 for (int e = w * HALF; e < (w + 1) * HALF; e += 4)
