@@ -22,7 +22,7 @@
  *   lse[b,h,i] = log(exp(sink_weights[h]) + sum_allowed exp(z_j))  (no sink term when NULL)
  *   out[b,h,i,:] = sum_allowed exp(z_j - lse) * v[b,g,j,:]
  * sliding_window counts the tokens a query sees including itself (the
- * forward's "number of causal tokens available to each query"); the page's
+ * forward describes it as a count of causal tokens per query); the page's
  * sliding-window mask mod (q_idx - kv_idx <= window) is sliding_window =
  * window + 1. The page applies `scale` when sink_weights is not set: with
  * sink weights the scale is head_dim^-0.5, and scale <= 0 also means

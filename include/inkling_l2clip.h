@@ -5,11 +5,12 @@
  * The operation is the per-head clipping that Inkling2 applies to q and k
  * ahead of the attention, as documented on the NVIDIA NeMo AutoModel API page
  * "nemo_automodel.components.models.inkling2.layers": L2Clip(heads, width,
- * threshold, learned_scale), "per-head L2 clipping, optionally preceded by
- * learned per-channel scales", and L2Clip.forward(x [batch, sequence, heads,
- * head_dim], tau [batch, sequence]), "clip head vectors, then apply optional
- * length scaling", the result in x's dtype. The page prints no formula; the
- * library computes the plainest reading, per (b, s, h) vector:
+ * threshold, learned_scale) clips each head's vector by its L2 norm, with
+ * optional learned per-channel scales before the clip, and L2Clip.forward(x
+ * [batch, sequence, heads, head_dim], tau [batch, sequence]) applies the
+ * optional tau as a length scaling after the clip and returns x's dtype. The
+ * page prints no formula; the library computes the plainest reading, per
+ * (b, s, h) vector:
  *   z = x * scale[h, :]                       (scale NULL: z = x)
  *   y = z * min(1, threshold / ||z||_2) * tau[b, s]   (tau NULL: no length scaling)
  * in FP32, y rounded to BF16 (round to nearest even).

@@ -11,8 +11,9 @@
  *     note that no sequence-by-sequence bias tensor is built and that
  *     gradients reach the profiles and the returned log-sum-exp;
  *   - "nemo_automodel.components.models.inkling2.attention",
- *     Inkling2Attention.forward ("zero-valued virtual sink") and the quadratic
- *     reference Inkling2Attention._eager ("without mutating inputs").
+ *     Inkling2Attention.forward (the sink as a virtual key whose value row is
+ *     zero) and the quadratic reference Inkling2Attention._eager (which leaves
+ *     its inputs untouched).
  *
  * Definition (b batch, h query head, g = h / (Hq/Hkv) its KV head, i local
  * query row, i_g = query_offset + i its global column, j key column):
@@ -91,9 +92,9 @@ size_t inkling_rel_attn_workspace_size(const inkling_rel_attn_dims* dims, int ba
  *   valid [B,S], key_valid [B,Skv] (uint8 0/1; key_valid NULL = valid, needs
  *   Skv == S and query_offset == 0), positions [B,S], key_positions [B,Skv]
  *   (int32; NULL defaults as in fwd).
- * Conditions (the page's "each batch row has a local slice of one global
- * contiguous real-token span", "global real-token positions are consecutive",
- * positions "reset per document"):
+ * Conditions (from the forward's argument notes: every batch row holds a slice
+ * of one contiguous run of real tokens, their global positions are consecutive,
+ * and positions restart at each document):
  *   - the valid columns of each row form one contiguous span (same for key_valid);
  *   - along valid columns each position is the previous one plus one, or 0
  *     (a new document); valid positions are >= 0;

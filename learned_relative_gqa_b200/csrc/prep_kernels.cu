@@ -12,7 +12,7 @@
 //   lo = max(i_g - positions[i], first valid key, i_g - W + 1 if W > 0)
 //   hi = min(i_g, last valid key)
 // i_g - positions[i] is the column where the row's document starts
-// ("positions ... reset per document" on the Inkling2FlexAttention.forward
+// (positions restart at every document, per the Inkling2FlexAttention.forward
 // page), so the interval is exactly the causal, same-document, in-window,
 // valid keys of the definition.
 #include <cuda_runtime.h>

@@ -22,9 +22,9 @@ Readings where the page leaves a point open (the CUDA path encodes the same):
   [kF, (k + 1)F) (the last one may be shorter); a query sees only keys of its
   own block. The rule is combined (AND) with the mask type.
 * F3 sliding_window W > 0: a query sees the W most recent tokens including
-  itself (i - j < W), which is the forward's "number of causal tokens
-  available to each query"; the mask mod's "q_idx - kv_idx <= window" is the
-  same rule with W + 1. W = 0: the full causal history.
+  itself (i - j < W), as the forward describes the parameter (a count of
+  causal tokens per query); the mask mod's inclusive bound q_idx - kv_idx <=
+  window is the same rule with W + 1. W = 0: the full causal history.
 * F4 sink_weights [Hq]: one logit per query head, acting as a virtual key
   with a zero value row in every row's softmax denominator; None = no sink.
 * F5 scale: the page applies ``scale`` when sink_weights is not set; with

@@ -6,10 +6,10 @@ CPU-baseline leg are the only callers; the product path never imports it.
 
 Follows the NeMo AutoModel API page for
 ``nemo_automodel.components.models.inkling2.layers``: ``L2Clip(heads, width,
-threshold, learned_scale)`` -- "per-head L2 clipping, optionally preceded by
-learned per-channel scales" -- and ``L2Clip.forward(x [batch, sequence, heads,
-head_dim], tau [batch, sequence] | None)`` -- "clip head vectors, then apply
-optional length scaling", tau "applied after clipping", result in x's dtype.
+threshold, learned_scale)`` clips each head's vector by its L2 norm, with
+optional learned per-channel scales in front, and ``L2Clip.forward(x [batch,
+sequence, heads, head_dim], tau [batch, sequence] | None)`` applies tau as a
+length scaling after the clip and returns x's dtype.
 
 The page names the operation but prints no formula; this module takes the
 plainest reading (the CUDA path encodes the same):

@@ -9,8 +9,8 @@
  * "nemo_automodel.components.models.inkling2.flex_attention" -- class
  * Inkling2FlexAttention and its forward() parameter list -- and
  * "nemo_automodel.components.models.inkling2.attention" -- the quadratic
- * reference Inkling2Attention._eager and the "zero-valued virtual sink" of
- * Inkling2Attention.forward):
+ * reference Inkling2Attention._eager and the sink of Inkling2Attention.forward,
+ * a virtual key whose value row is zero):
  *
  *   For every batch b, query head h (kv head g = h / (Hq/Hkv)) and local query
  *   row i (global column i_g = query_offset + i), over the keys j that are
@@ -27,10 +27,10 @@
  * Readings taken where the pages are silent (each is listed in the design
  * notes): the sink is a virtual key with logit sink[b,i,h] and a zero value
  * row; lse includes the sink; a query row with no allowed key has out = 0 and
- * lse = sink; "reset per document" means two tokens share a document exactly
+ * lse = sink; positions restarting per document means two tokens share one exactly
  * when their logical-position difference equals their column difference; the
  * window admits i_g - j < W (W tokens including the query itself) unless the
- * caller asks for the generic FlexAttention docstring's "<= W" reading through
+ * caller asks for the generic FlexAttention docstring's inclusive reading through
  * window_inclusive (only a self-test uses that).
  *
  * The backward pass is the chain rule of the formulas above, written out

@@ -5,7 +5,9 @@ closed forms derived by hand, torch library routines on a differently written
 dense formulation (tests/dense_reference.py), invariants the mathematics fixes,
 and finite differences of the oracle's own forward for its backward.
 """
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -57,6 +59,9 @@ def mask_of(x):
                             heads_q=x["q"].shape[2])
 
 
+GOLDEN = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_closed_form.json")))
+
+
 def tiny_case(R, sink1=None):
     """The hand-worked case: B=1, S=2, H=1, D=1 (scale 1), positions [0,1]."""
     s1 = np.float32(math.log(2.0)) if sink1 is None else sink1
@@ -85,9 +90,11 @@ def test_tiny_closed_form_forward():
     np.testing.assert_allclose(out.ravel(), [out0, out1], rtol=1e-13)
     np.testing.assert_allclose(lse.ravel(), [lse0, lse1], rtol=1e-13)
     np.testing.assert_allclose(lsec.ravel(), [z00, math.log(math.exp(z10) + math.exp(z11))], rtol=1e-13)
-    # the values quoted in the hand derivation
+    # the values quoted in the hand derivation, and the stored fixture of the same case
     np.testing.assert_allclose(out.ravel(), [1.635148952, 1.807489729], atol=2e-9)
     np.testing.assert_allclose(lse.ravel(), [1.701413278, 2.340752954], atol=2e-9)
+    np.testing.assert_allclose(out.ravel(), GOLDEN["R2"]["out"], rtol=1e-13)
+    np.testing.assert_allclose(lse.ravel(), GOLDEN["R2"]["lse"], rtol=1e-13)
 
 
 def test_tiny_closed_form_no_bias_beyond_extent():
@@ -100,6 +107,8 @@ def test_tiny_closed_form_no_bias_beyond_extent():
     np.testing.assert_allclose(out.ravel()[1], out1, rtol=1e-13)
     np.testing.assert_allclose(lse.ravel()[1], lse1, rtol=1e-13)
     np.testing.assert_allclose([out.ravel()[1], lse.ravel()[1]], [1.650244591, 1.743668381], atol=2e-9)
+    np.testing.assert_allclose([out.ravel()[1], lse.ravel()[1]], [GOLDEN["R1_row1"]["out"], GOLDEN["R1_row1"]["lse"]],
+                               rtol=1e-13)
 
 
 def test_tiny_closed_form_plain_causal_softmax():
@@ -111,6 +120,8 @@ def test_tiny_closed_form_plain_causal_softmax():
     e = math.e
     np.testing.assert_allclose(out.ravel(), [2.0, (2 * e + 4) / (e + 1)], rtol=1e-13)
     np.testing.assert_allclose(lse.ravel(), [1.0, math.log(e + 1)], rtol=1e-13)
+    np.testing.assert_allclose(out.ravel(), GOLDEN["plain_causal_zero_profiles_no_sink"]["out"], rtol=1e-13)
+    np.testing.assert_allclose(lse.ravel(), GOLDEN["plain_causal_zero_profiles_no_sink"]["lse"], rtol=1e-13)
 
 
 def test_tiny_closed_form_backward():
@@ -142,6 +153,9 @@ def test_tiny_closed_form_backward():
     dp = g["dprofiles"].reshape(2, 2)
     np.testing.assert_allclose([dp[0, 0], dp[1, 1], dp[1, 0]], [0.298292904, 0.136919964, 0.211040373],
                                atol=2e-9)
+    gb = GOLDEN["R2_backward_dout_ones"]
+    np.testing.assert_allclose(g["dsink"].ravel(), gb["dsink"], rtol=1e-12)
+    np.testing.assert_allclose([dp[0, 0], dp[1, 1], dp[1, 0]], gb["dprofiles_00_11_10"], rtol=1e-12)
 
 
 def test_empty_row_gives_zero_output_and_sink_lse():
