@@ -16,6 +16,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "inkling_l2clip.h"
 
@@ -269,6 +270,14 @@ inkling_status check(const inkling_l2clip_dims* d) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A named NVTX range over an entry point (a no-op when no profiler is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 inkling_status status_of(cudaError_t e) { return ira::note_cuda_error(e) == cudaSuccess ? INKLING_OK : INKLING_ERR_CUDA; }
 
 }  // namespace
@@ -282,6 +291,7 @@ size_t inkling_l2clip_workspace_size(const inkling_l2clip_dims* dims) {
 
 inkling_status inkling_l2clip_fwd(const inkling_l2clip_dims* dims, const uint16_t* x, const float* scale,
                                   const float* tau, uint16_t* y, void* stream) {
+    NvtxRange nvtx_range("inkling_l2clip_fwd");
     inkling_status s = check(dims);
     if (s != INKLING_OK) return s;
     const int64_t rows = dims->batch * dims->seq * dims->heads;
@@ -303,6 +313,7 @@ inkling_status inkling_l2clip_fwd(const inkling_l2clip_dims* dims, const uint16_
 inkling_status inkling_l2clip_bwd(const inkling_l2clip_dims* dims, const uint16_t* x, const float* scale,
                                   const float* tau, const float* dy, float* dx, float* dscale, float* dtau,
                                   void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("inkling_l2clip_bwd");
     inkling_status s = check(dims);
     if (s != INKLING_OK) return s;
     if ((scale == nullptr) != (dscale == nullptr) || (tau == nullptr) != (dtau == nullptr))
