@@ -29,9 +29,14 @@
  * Conventions for every entry point:
  *   - All tensors are dense, row-major, in device memory owned by the caller.
  *     BF16 tensors are passed as their 16-bit patterns (uint16_t).
- *   - The library allocates no memory and keeps no state between calls;
- *     scratch lives in a caller-provided device workspace whose size comes from
- *     inkling_rel_attn_workspace_size(). Inputs are never written.
+ *   - The library allocates no device memory; scratch lives in a
+ *     caller-provided device workspace whose size comes from
+ *     inkling_rel_attn_workspace_size(). Inputs are never written. The only
+ *     state kept between calls is, per host thread and device, one non-blocking
+ *     CUDA stream and four events, created by the first backward call made
+ *     outside a stream capture and reused: the backward forks part of its work
+ *     onto that stream and joins it back to `stream` with the events before it
+ *     returns, so all of it is ordered on `stream` (and captured with it).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   - Argument errors are detected on the host before anything is launched and
  *     returned synchronously. fwd/bwd are asynchronous: a device-side failure
