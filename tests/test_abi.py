@@ -174,3 +174,35 @@ def test_l2clip_rejects_bad_arguments_on_host(lib):
     assert lib.inkling_l2clip_bwd(ctypes.byref(good), fake, None, None, fake, fake, None, fake, fake, 1 << 30,
                                   None) == 1
     assert lib.inkling_l2clip_bwd(ctypes.byref(good), fake, None, None, fake, fake, None, None, fake, 16, None) == 1
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No CPU or library fallback: a missing shared library raises on load."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from learned_relative_gqa_b200 import binding\n"
+            "binding._lib = None\n"
+            "try:\n"
+            "    binding.load(%r)\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n"
+            "else:\n"
+            "    print('loaded')\n") % (ROOT, str(tmp_path / "libinkling_rel_attn.so"))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.startswith("raised:") and "not built" in r.stdout
+
+
+def test_product_modules_do_not_import_the_oracle():
+    import ast
+    pkg = os.path.join(ROOT, "learned_relative_gqa_b200")
+    for name in os.listdir(pkg):
+        if not name.endswith(".py"):
+            continue
+        tree = ast.parse(open(os.path.join(pkg, name)).read())
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                assert all(not a.name.startswith("oracle") for a in node.names), name
+            elif isinstance(node, ast.ImportFrom):
+                assert not (node.module or "").startswith("oracle"), name
