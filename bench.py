@@ -540,7 +540,12 @@ def main():
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
     ms_step = ms_max / args.steps
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    # every rank draws its own documents, so the job's FLOPs are the sum over ranks
+    fl_t = torch.tensor([flops_step], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(fl_t, op=dist.ReduceOp.SUM)
+    flops_job = float(fl_t.item())
+    value = flops_job / (ms_step * 1e-3) / 1e12
 
     # per-kernel durations (events recorded on the launch stream around each kernel)
     kt = per_kernel_times(buf, args.steps, backward)
@@ -578,7 +583,7 @@ def main():
         e_t = torch.tensor([e_ms], device=device, dtype=torch.float64)
         if dist is not None:
             dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": flops_step * world / (float(e_t.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": flops_job / (float(e_t.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(float(e_t.item()), 3),
                "overlap": "copy-in, kernels and copy-out of consecutive steps on three streams, two buffer sets"}
 
