@@ -725,6 +725,8 @@ def run_config(w, x, E, flops_step, world):
                          f"W{w.window} R{w.rel_extent} docs{w.docs} pad{w.pad}, {'fwd+bwd' if w.backward else 'fwd'}"),
             "global_batch": w.batch * world, "seq_len": w.seq, "parallelism": f"replicas x{world}",
             "allowed_elements": E, "flops_per_step": flops_step,
+            "counts": ("allowed_elements and flops_per_step are one rank's batch; each rank draws its own "
+                       "documents and value sums the FLOPs of all ranks" if world > 1 else "one GPU"),
             "l2": "inputs larger than L2 (profiles %.2f GB/step)" % (x["profiles"].numel() * 2 / 1e9)}
 
 
