@@ -465,6 +465,17 @@ def e2e_run(x, steps, backward):
     return ms / steps, h2d, d2h
 
 
+def spawn_ranks(n: int) -> int:
+    """Re-runs this command under torch.distributed.run with n ranks on this node."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -488,6 +499,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "ours" and world != args.gpus:
+        if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+            # not started by a launcher: start one rank per GPU on this node and pass
+            # their exit status through (rank 0 prints the JSON line)
+            sys.exit(spawn_ranks(args.gpus))
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU", file=sys.stderr)
+        sys.exit(2)
     from learned_relative_gqa_b200 import workloads
     import dataclasses
     w = workloads.BY_NAME[args.workload]

@@ -60,6 +60,51 @@ inkling_status inkling_l2clip_bwd(const inkling_l2clip_dims* dims, const uint16_
                                   const float* tau, const float* dy, float* dx, float* dscale, float* dtau,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * L2Clip of q fused into the learned-relative attention (inkling_rel_attn.h): the
+ * clipping Inkling2 applies to q ahead of the attention (the q_l2_clip attribute of
+ * Inkling2Attention on the "nemo_automodel.components.models.inkling2.attention"
+ * page; L2Clip.forward(x, tau) on the "...inkling2.layers" page), done inside the
+ * attention kernels instead of as a pass of its own. Same arithmetic as
+ * inkling_l2clip_fwd / _bwd above with H = heads_q, D = head_dim:
+ *
+ * inkling_rel_attn_fwd_qclip: x [B,S,Hq,D] BF16 is the unclipped q. Each query tile
+ *   is clipped in shared memory as soon as it is loaded, y = z min(1, threshold /
+ *   |z|) tau (z = x * clip_scale), rounded to BF16, and used for the attention; y is
+ *   also stored to q_clipped [B,S,Hq,D] BF16 for the backward. Every other argument
+ *   and result as in inkling_rel_attn_fwd.
+ * inkling_rel_attn_bwd_qclip: takes x and the forward's q_clipped; the attention
+ *   gradients are those of inkling_rel_attn_bwd with q = q_clipped, except that the
+ *   dQ kernel turns the query gradient into the gradient of x through the clip
+ *   (written to dx [B,S,Hq,D] FP32), and writes the parts of dclip_scale [Hq,D] and
+ *   dtau [B,S] that a final fixed-order sum adds up (each NULL exactly when its
+ *   parameter is NULL).
+ * clip_scale [Hq,D] and tau [B,S] FP32 or NULL; threshold >= 0 and finite.
+ * Workspace: inkling_rel_attn_qclip_workspace_size(dims, backward) bytes (the
+ * forward's equals inkling_rel_attn_workspace_size's). Errors as in the unfused
+ * calls, plus INKLING_ERR_INVALID_ARG for a bad threshold or a NULL q_clipped / x.
+ * Both asynchronous on `stream`.
+ */
+size_t inkling_rel_attn_qclip_workspace_size(const inkling_rel_attn_dims* dims, int backward);
+
+inkling_status inkling_rel_attn_fwd_qclip(const inkling_rel_attn_dims* dims, double threshold,
+                                          const float* clip_scale, const float* tau, const uint16_t* x,
+                                          const uint16_t* k, const uint16_t* v, const uint16_t* profiles,
+                                          const float* sink, const uint8_t* valid, const uint8_t* key_valid,
+                                          const int32_t* positions, const int32_t* key_positions,
+                                          uint16_t* q_clipped, float* out, float* lse, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+inkling_status inkling_rel_attn_bwd_qclip(const inkling_rel_attn_dims* dims, double threshold,
+                                          const float* clip_scale, const float* tau, const uint16_t* x,
+                                          const uint16_t* q_clipped, const uint16_t* k, const uint16_t* v,
+                                          const uint16_t* profiles, const float* sink, const uint8_t* valid,
+                                          const uint8_t* key_valid, const int32_t* positions,
+                                          const int32_t* key_positions, const float* out, const float* lse,
+                                          const float* dout, const float* dlse, float* dx, float* dk, float* dv,
+                                          float* dprofiles, float* dsink, float* dclip_scale, float* dtau,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

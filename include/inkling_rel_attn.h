@@ -31,12 +31,16 @@
  *     BF16 tensors are passed as their 16-bit patterns (uint16_t).
  *   - The library allocates no device memory; scratch lives in a
  *     caller-provided device workspace whose size comes from
- *     inkling_rel_attn_workspace_size(). Inputs are never written. The only
- *     state kept between calls is, per host thread and device, one non-blocking
+ *     inkling_rel_attn_workspace_size(). Inputs are never written. The state
+ *     kept between calls is, per host thread and device, one non-blocking
  *     CUDA stream and four events, created by the first backward call made
  *     outside a stream capture and reused: the backward forks part of its work
  *     onto that stream and joins it back to `stream` with the events before it
  *     returns, so all of it is ordered on `stream` (and captured with it).
+ *     One exception: inkling_rel_attn_fwd_noalloc takes no workspace; its
+ *     scratch is a static device array inside the library that keeps the last
+ *     call's contents, and the library caches that array's address per CUDA
+ *     context (see that entry point).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   - Argument errors are detected on the host before anything is launched and
  *     returned synchronously. fwd/bwd are asynchronous: a device-side failure
@@ -169,9 +173,13 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims,
  *   - Every call on a device shares the array and it keeps the last call's
  *     contents: calls that overlap on the GPU (other streams, other host
  *     threads) race on it, so serialise them.
- *   - A device-side wait that runs out is recorded inside that array, which
- *     callers cannot hand to inkling_rel_attn_last_device_error; the outputs of
- *     such a call are unspecified.
+ *   - The address is cached per CUDA context (by the context's
+ *     process-unique id), so a context created after cudaDeviceReset, or a
+ *     non-primary context the caller made current, gets its own lookup; that
+ *     lookup is again a first call and belongs before any stream capture.
+ *   - A device-side wait that runs out is recorded at the start of that array;
+ *     inkling_rel_attn_fwd_noalloc_last_device_error() reads (and clears) it.
+ *     The outputs of such a call are unspecified.
  */
 inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims,
                                             const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -180,10 +188,34 @@ inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims,
                                             const int32_t* positions, const int32_t* key_positions,
                                             float* out, float* lse, void* stream);
 
+/*
+ * Context parallelism (the forward's query_offset / key_valid / key_positions
+ * arguments, whose key side is global under CP, on the Inkling2FlexAttention
+ * page): merges a second result for the same query rows, computed over a key
+ * set disjoint from the first one, into the first (ASYNCHRONOUS on stream):
+ *   lse = log(exp(lse) + exp(lse_part))
+ *   out = out * exp(lse_old - lse) + out_part * exp(lse_part - lse)
+ * out, out_part: [rows, head_dim] fp32 (rows = B * S * Hq, 16-byte aligned);
+ * lse, lse_part: [rows] fp32, natural log. out / lse are updated in place; the
+ * sink must be counted in exactly one of the two parts (the other passes a sink
+ * of -inf). A row with both lse at -inf stays out = 0, lse = -inf.
+ * head_dim 64 or 128; INKLING_ERR_INVALID_ARG for null or misaligned pointers.
+ */
+inkling_status inkling_rel_attn_merge(int64_t rows, int64_t head_dim, float* out, float* lse,
+                                      const float* out_part, const float* lse_part, void* stream);
+
 /* SYNCHRONOUS: waits on stream, returns INKLING_ERR_TIMEOUT if a kernel of the
  * last fwd/bwd call on this workspace gave up a bounded wait (and clears the
  * record), INKLING_OK otherwise. */
 inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream);
+
+/* SYNCHRONOUS: the same check for inkling_rel_attn_fwd_noalloc, whose device
+ * error word lives in the library's static scratch array of the current CUDA
+ * context: waits on stream, returns INKLING_ERR_TIMEOUT if a kernel of the last
+ * no-allocation forward gave up a bounded wait (and clears the record),
+ * INKLING_OK otherwise. Like that entry point, it allocates nothing and has no
+ * counterpart on the Inkling2 pages. */
+inkling_status inkling_rel_attn_fwd_noalloc_last_device_error(void* stream);
 
 /* Diagnostic: runs one kernel whose bounded wait is on an mbarrier that nothing
  * arrives on, with a limit of `timeout_us` microseconds, and returns the
@@ -191,6 +223,17 @@ inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream)
  * SYNCHRONOUS. Needs 16 bytes of workspace. */
 inkling_status inkling_rel_attn_selftest_wait_timeout(uint32_t timeout_us, void* workspace,
                                                       size_t workspace_bytes, void* stream);
+
+/* Diagnostic: sets the limit of the attention kernels' pipeline waits (every wait
+ * of a CTA on its copies, its tensor-core products and its other warps) for the
+ * fwd / bwd calls that follow, in nanoseconds; 0 restores the default (2 s).
+ * When a wait runs out, the CTA records the site in the workspace's error word
+ * (read by inkling_rel_attn_last_device_error), stops, and drains what it has in
+ * flight before it exits; those drain waits always keep the default limit.
+ * Limits below 20 us are polled without sleeping, so a limit of 1 ns makes every
+ * wait that does not succeed at its first test run out (a CTA's first wait, for
+ * its Q tile, always does) and exercises that path. Host-side, not thread-safe. */
+inkling_status inkling_rel_attn_set_wait_timeout_ns(uint64_t timeout_ns);
 
 /* Diagnostic: evaluates, on the device, the FMA-pipe power of two the forward
  * kernel uses for a share of its softmax exponentials (range reduction

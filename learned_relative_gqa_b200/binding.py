@@ -77,12 +77,18 @@ def load(path: str = LIB_PATH):
     lib.inkling_rel_attn_bwd.argtypes = [dp] + [vp] * 18 + [vp, sz, vp]
     lib.inkling_rel_attn_fwd_noalloc.restype = ctypes.c_int
     lib.inkling_rel_attn_fwd_noalloc.argtypes = [dp] + [vp] * 11 + [vp]
+    lib.inkling_rel_attn_fwd_noalloc_last_device_error.restype = ctypes.c_int
+    lib.inkling_rel_attn_fwd_noalloc_last_device_error.argtypes = [vp]
+    lib.inkling_rel_attn_merge.restype = ctypes.c_int
+    lib.inkling_rel_attn_merge.argtypes = [ctypes.c_int64, ctypes.c_int64, vp, vp, vp, vp, vp]
     lib.inkling_rel_attn_last_device_error.restype = ctypes.c_int
     lib.inkling_rel_attn_last_device_error.argtypes = [vp, vp]
     lib.inkling_rel_attn_selftest_exp2.restype = ctypes.c_int
     lib.inkling_rel_attn_selftest_exp2.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.inkling_rel_attn_selftest_wait_timeout.restype = ctypes.c_int
     lib.inkling_rel_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
+    lib.inkling_rel_attn_set_wait_timeout_ns.restype = ctypes.c_int
+    lib.inkling_rel_attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.inkling_rel_attn_set_timing_events.restype = ctypes.c_int
     lib.inkling_rel_attn_set_timing_events.argtypes = [vp, ctypes.c_int]
     fd = ctypes.POINTER(FlexDims)
@@ -99,6 +105,12 @@ def load(path: str = LIB_PATH):
     lib.inkling_l2clip_fwd.argtypes = [ld] + [vp] * 4 + [vp]
     lib.inkling_l2clip_bwd.restype = ctypes.c_int
     lib.inkling_l2clip_bwd.argtypes = [ld] + [vp] * 7 + [vp, sz, vp]
+    lib.inkling_rel_attn_qclip_workspace_size.restype = sz
+    lib.inkling_rel_attn_qclip_workspace_size.argtypes = [dp, ctypes.c_int]
+    lib.inkling_rel_attn_fwd_qclip.restype = ctypes.c_int
+    lib.inkling_rel_attn_fwd_qclip.argtypes = [dp, ctypes.c_double] + [vp] * 14 + [vp, sz, vp]
+    lib.inkling_rel_attn_bwd_qclip.restype = ctypes.c_int
+    lib.inkling_rel_attn_bwd_qclip.argtypes = [dp, ctypes.c_double] + [vp] * 23 + [vp, sz, vp]
     lib.inkling_rel_attn_last_cuda_error.restype = ctypes.c_char_p
     lib.inkling_rel_attn_last_cuda_error.argtypes = []
     lib.inkling_status_string.restype = ctypes.c_char_p
@@ -186,6 +198,22 @@ def inkling_rel_attn_fwd_noalloc(dims: Dims, q, k, v, profiles, sink, valid, key
         _p(positions), _p(key_positions), _p(out), _p(lse), _stream(stream)))
 
 
+def inkling_rel_attn_merge(out, lse, out_part, lse_part, stream=None) -> None:
+    """Merges (out_part, lse_part), a result over a disjoint key set, into (out, lse) in place."""
+    for t in (out, lse, out_part, lse_part):
+        if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()):
+            raise ValueError("inkling_rel_attn_merge: contiguous float32 CUDA tensors expected")
+    if out.shape != out_part.shape or lse.shape != lse_part.shape or out.shape[:-1] != lse.shape:
+        raise ValueError("inkling_rel_attn_merge: shape mismatch")
+    _check(load().inkling_rel_attn_merge(int(lse.numel()), int(out.shape[-1]), _p(out), _p(lse), _p(out_part),
+                                         _p(lse_part), _stream(stream)), "inkling_rel_attn_merge")
+
+
+def inkling_rel_attn_fwd_noalloc_last_device_error(stream=None) -> int:
+    """Reads and clears the device error word of the no-allocation forward (synchronous)."""
+    return int(load().inkling_rel_attn_fwd_noalloc_last_device_error(_stream(stream)))
+
+
 def inkling_rel_attn_last_device_error(workspace, stream=None) -> int:
     return int(load().inkling_rel_attn_last_device_error(_p(workspace), _stream(stream)))
 
@@ -193,6 +221,11 @@ def inkling_rel_attn_last_device_error(workspace, stream=None) -> int:
 def inkling_rel_attn_selftest_wait_timeout(timeout_us: int, workspace, stream=None) -> int:
     return int(load().inkling_rel_attn_selftest_wait_timeout(int(timeout_us), _p(workspace), workspace.numel(),
                                                              _stream(stream)))
+
+
+def inkling_rel_attn_set_wait_timeout_ns(timeout_ns: int) -> None:
+    """Limit of the attention kernels' pipeline waits for later calls (0 = default)."""
+    _check(load().inkling_rel_attn_set_wait_timeout_ns(int(timeout_ns)), "inkling_rel_attn_set_wait_timeout_ns")
 
 
 def inkling_rel_attn_selftest_exp2(t, out, stream=None) -> None:
@@ -243,6 +276,55 @@ def backward(q, k, v, profiles, sink, valid, key_valid, positions, key_positions
     inkling_rel_attn_bwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout,
                          dlse, dq, dk, dv, dprof, dsink, ws, stream)
     return dict(dq=dq, dk=dk, dv=dv, dprofiles=dprof, dsink=dsink)
+
+
+# --------------------------------------------------------------------------
+# L2Clip of q fused into the attention (include/inkling_l2clip.h, *_qclip)
+# --------------------------------------------------------------------------
+def forward_qclip(x, k, v, profiles, sink, valid, key_valid=None, positions=None, key_positions=None, *,
+                  threshold: float, clip_scale=None, tau=None, window: int = 0, query_offset: int = 0,
+                  workspace=None, stream=None):
+    """out [B,S,Hq,D] fp32, lse [B,S,Hq] fp32 and the clipped q [B,S,Hq,D] BF16 of the
+    attention with q = L2Clip(x) computed inside the kernels."""
+    _contig(x, k, v, profiles, sink, valid, key_valid, positions, key_positions, clip_scale, tau)
+    dims = make_dims(x, k, profiles, window, query_offset)
+    out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    lse = torch.empty(x.shape[:3], dtype=torch.float32, device=x.device)
+    qc = torch.empty_like(x)
+    if workspace is None:
+        workspace = torch.empty(max(int(load().inkling_rel_attn_qclip_workspace_size(ctypes.byref(dims), 0)), 256),
+                                dtype=torch.uint8, device=x.device)
+    st = load().inkling_rel_attn_fwd_qclip(
+        ctypes.byref(dims), float(threshold), _p(clip_scale), _p(tau), _p(x), _p(k), _p(v), _p(profiles), _p(sink),
+        _p(_u8(valid)), _p(_u8(key_valid)), _p(positions), _p(key_positions), _p(qc), _p(out), _p(lse),
+        _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_rel_attn_fwd_qclip")
+    return out, lse, qc
+
+
+def backward_qclip(x, q_clipped, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout,
+                   dlse=None, *, threshold: float, clip_scale=None, tau=None, window: int = 0, query_offset: int = 0,
+                   workspace=None, stream=None):
+    """dict dx (gradient of the unclipped q), dk, dv, dprofiles, dsink, dclip_scale, dtau (fp32;
+    the last two None without their parameters)."""
+    _contig(x, q_clipped, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout, dlse,
+            clip_scale, tau)
+    dims = make_dims(x, k, profiles, window, query_offset)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = dict(dx=torch.empty(x.shape, **f32), dk=torch.empty(k.shape, **f32), dv=torch.empty(v.shape, **f32),
+             dprofiles=torch.empty(profiles.shape, **f32), dsink=torch.empty(sink.shape, **f32),
+             dclip_scale=None if clip_scale is None else torch.empty(clip_scale.shape, **f32),
+             dtau=None if tau is None else torch.empty(tau.shape, **f32))
+    if workspace is None:
+        workspace = torch.empty(int(load().inkling_rel_attn_qclip_workspace_size(ctypes.byref(dims), 1)),
+                                dtype=torch.uint8, device=x.device)
+    st = load().inkling_rel_attn_bwd_qclip(
+        ctypes.byref(dims), float(threshold), _p(clip_scale), _p(tau), _p(x), _p(q_clipped), _p(k), _p(v),
+        _p(profiles), _p(sink), _p(_u8(valid)), _p(_u8(key_valid)), _p(positions), _p(key_positions), _p(out),
+        _p(lse), _p(dout), _p(dlse), _p(g["dx"]), _p(g["dk"]), _p(g["dv"]), _p(g["dprofiles"]), _p(g["dsink"]),
+        _p(g["dclip_scale"]), _p(g["dtau"]), _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "inkling_rel_attn_bwd_qclip")
+    return g
 
 
 # --------------------------------------------------------------------------

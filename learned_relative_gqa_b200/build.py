@@ -15,6 +15,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libinkling_rel_attn.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
+# the same kernels with every shared / global index checked (-DINKLING_BOUNDS_CHECK), for tests
+BOUNDS_CHECK_LIB_PATH = os.path.join(HERE, "libinkling_rel_attn_boundscheck.so")
 SOURCES = ["host.cu", "prep_kernels.cu", "fwd.cu", "bwd.cu", "l2clip.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -26,12 +28,16 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def stale(path: str = LIB_PATH) -> bool:
+    """True when the library at `path` is missing or older than a source or header."""
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     return any(os.path.getmtime(d) > t for d in deps)
+
+
+_stale = stale
 
 
 def build(force: bool = False, verbose: bool = False, out_path: str = LIB_PATH, defines: tuple = ()) -> str:
@@ -47,11 +53,14 @@ def build(force: bool = False, verbose: bool = False, out_path: str = LIB_PATH, 
     if verbose:
         common += ["-Xptxas", "-v"]
     common += [f"-D{d}" for d in defines]
-    for src in SOURCES:
+    procs = []
+    for src in SOURCES:  # translation units compile side by side
         obj = os.path.join(build_dir, src.replace(".cu", ".o"))
-        cmd = common + ["-c", os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
+        procs.append((subprocess.Popen(common + ["-c", os.path.join(CSRC, src), "-o", obj]), src))
         objs.append(obj)
+    failed = [src for proc, src in procs if proc.wait() != 0]
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
     tmp = out_path + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, out_path)

@@ -44,7 +44,8 @@ namespace kv {
 
 constexpr int BK = 128;              // keys per CTA (TMEM lanes)
 constexpr int BQ = 64;               // queries per step
-constexpr int HALF = BQ / 2;         // query columns per elementwise warpgroup
+constexpr int NWG = 4;               // elementwise warpgroups
+constexpr int COLS = BQ / NWG;       // query columns per elementwise warpgroup
 constexpr int BAND_LEN = 136;        // bf16 per band row: 128 distances + up to 7 of misalignment
 constexpr int BAND_PITCH = BAND_LEN * 2;
 // Band rows of a step, fetched as 9 TMA boxes of 8 rows (2176 B each, so every box
@@ -86,16 +87,24 @@ struct Layout {
     static constexpr uint32_t s_col(int bb) { return uint32_t(2 * D + 128 * bb); }
     static constexpr uint32_t dp_col(int bb) { return uint32_t(2 * D + 128 * bb + 64); }
     static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int NWARPS = 4 * NWG + 4;
+    // registers per thread at launch, and after the split: control warpgroup / elementwise
+    static constexpr int REG_LAUNCH = 96, REG_CTRL = 56, REG_EW = 104;
+    static_assert(128 * REG_CTRL + 128 * NWG * REG_EW <= 32 * NWARPS * REG_LAUNCH, "register split");
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    // the epilogue stages 32 x 32 chunks of every warp through the K, V, Q and dO tiles
+    static_assert(4 * NWG * 32 * 36 * 4 <= BAND_OFF - K_OFF, "epilogue staging");
 };
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_band, const AttnParams p, const int num_ktiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9, BAND_WARP = 10, MMA_WARP_B = 11;
+    constexpr int CTRL = 4 * NWG;
+    constexpr int TMA_WARP = CTRL, MMA_WARP = CTRL + 1, BAND_WARP = CTRL + 2, MMA_WARP_B = CTRL + 3;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
@@ -121,6 +130,9 @@ __global__ void __launch_bounds__(384, 1)
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int j0 = kt * BK;
     const int t64 = (p.S + 63) / 64;
+    // buffer extents for the bounds-checking build (elements; shared memory in bytes)
+    [[maybe_unused]] const uint32_t smem_base = smem_u32(smem);
+    [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -131,13 +143,13 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(&s_full[u], 2);
-            mbar_init(&p_full[u], 8);
+            mbar_init(&p_full[u], 4 * NWG);
         }
         mbar_init(acc_full, 2);
         mbar_init(drain, 2);
         for (int u = 0; u < NB; ++u) {
             mbar_init(&band_full[u], 1);
-            mbar_init(&band_empty[u], 8);  // every elementwise warp
+            mbar_init(&band_empty[u], 4 * NWG);  // every elementwise warp
         }
         ctl->abort = 0;
         tinfo[0] = 0x7FFFFFFF;  // first query tile that sees the key tile
@@ -152,6 +164,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     // query tiles whose allowed key ranges intersect [j0, j0 + BK)
     for (int t = threadIdx.x; t < t64; t += blockDim.x) {
+        if (!IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, size_t(b) * t64 + t, 1, (long long)p.B * t64)) continue;
         const TileBounds tb = p.tile_bounds[size_t(b) * t64 + t];
         if (tb.n_nonempty > 0 && tb.min_lo <= j0 + BK - 1 && tb.max_hi >= j0) {
             atomicMin(&tinfo[0], t);
@@ -172,13 +185,14 @@ __global__ void __launch_bounds__(384, 1)
     auto step_h = [&](int n) { return g * G + n / n_qt; };
     auto step_qt = [&](int n) { return qt_first + n % n_qt; };
 
-    // Launched with 384 x 168 registers; warpgroup 2 (tile producer, two MMA issuers,
-    // band producer) gives part of its share to the two elementwise warpgroups
-    // (128 x 72 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
+    // Launched with REG_LAUNCH registers per thread; the control warpgroup (tile producer,
+    // two MMA issuers, band producer) gives part of its share to the elementwise
+    // warpgroups (checked against the launch total in Layout). Each change sits at the
+    // top of its branch.
     // A step whose smallest distance delta - 127 is >= R has no profile entry.
     auto band_used = [&](int n) { return p.R > 0 && p.q_off + step_qt(n) * BQ - j0 - (BK - 1) < p.R; };
-    if (warp >= 8) {
-        setmaxnreg_dec<72>();
+    if (warp >= CTRL) {
+        setmaxnreg_dec<L::REG_CTRL>();
     if (warp == TMA_WARP) {
         if (lane == 0 && n_steps > 0) {
             prefetch_tensormap(&tm_q);
@@ -203,9 +217,9 @@ __global__ void __launch_bounds__(384, 1)
                 IRA_TRACE(p, 21, n);
                 last = n;
             }
-            mbar_wait_drain(kv_full, 0, p.timeout_ns);
+            mbar_wait_drain(kv_full, 0);
             for (int n = (last >= NST ? last - NST + 1 : 0); n <= last; ++n)
-                mbar_wait_drain(&qd_full[n % NST], (n / NST) & 1, p.timeout_ns);
+                mbar_wait_drain(&qd_full[n % NST], (n / NST) & 1);
         }
     } else if (warp == BAND_WARP) {
         // ------------------------------------------------------------ band producer
@@ -221,7 +235,8 @@ __global__ void __launch_bounds__(384, 1)
             float l2_r[2], dv_r[2];
             bool full_r = false;
             auto load_info = [&](int n) {
-                if (n < n_steps) {
+                if (n < n_steps &&
+                    IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, size_t(b) * t64 + step_qt(n), 1, (long long)p.B * t64)) {
                     const TileBounds tb = p.tile_bounds[size_t(b) * t64 + step_qt(n)];
                     full_r = tb.n_nonempty == BQ && tb.max_lo <= j0 && tb.min_hi >= j0 + BK - 1;
                 }
@@ -231,9 +246,11 @@ __global__ void __launch_bounds__(384, 1)
                     l2_r[k] = 0.f;
                     dv_r[k] = 0.f;
                     const int i = step_qt(n) * BQ + lane + 32 * k;
-                    if (n < n_steps && i < p.S) {
+                    const size_t t = (size_t(b) * p.Hq + step_h(n)) * p.S + i;
+                    if (n < n_steps && i < p.S &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, size_t(b) * p.S + i, 1, (long long)p.B * p.S) &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, t, 1, n_rows)) {
                         rb_r[k] = p.row_bounds[size_t(b) * p.S + i];
-                        const size_t t = (size_t(b) * p.Hq + step_h(n)) * p.S + i;
                         l2_r[k] = p.lse2t[t];
                         dv_r[k] = p.dvt[t];
                     }
@@ -246,6 +263,8 @@ __global__ void __launch_bounds__(384, 1)
                 if (!warp_wait(&band_empty[buf], ((n / NB) & 1) ^ 1, ctl, p.err, kErrDkdvQFree, p.timeout_ns)) break;
                 const int h = step_h(n), i0 = step_qt(n) * BQ;
                 StepInfo* info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF) + buf;
+                if (!IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, smem_u32(info) - smem_base, sizeof(StepInfo), L::TOTAL))
+                    info = reinterpret_cast<StepInfo*>(smem + L::INFO_OFF);
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     const int c = lane + 32 * k;
@@ -267,7 +286,10 @@ __global__ void __launch_bounds__(384, 1)
                         uint8_t* band = smem + L::BAND_OFF + buf * BAND_BYTES;
                         // box g: shared rows 8g .. 8g+7 = columns 8g - dm .. 8g - dm + 7
                         for (int g8 = 0; g8 < BAND_BOXES; ++g8)
-                            tma_load_2d(band + g8 * 8 * BAND_PITCH, &tm_band, &band_full[buf], x0 + 8 * g8, row0 + 8 * g8);
+                            if (IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, smem_u32(band + g8 * 8 * BAND_PITCH) - smem_base,
+                                              8 * BAND_PITCH, L::TOTAL))
+                                tma_load_2d(band + g8 * 8 * BAND_PITCH, &tm_band, &band_full[buf], x0 + 8 * g8,
+                                            row0 + 8 * g8);
                     }
                     IRA_TRACE(p, 34, n);
                 }
@@ -276,7 +298,7 @@ __global__ void __launch_bounds__(384, 1)
             // never leave a copy in flight into shared memory of an exiting CTA
             if (lane == 0)
                 for (int n = (last >= NB ? last - NB + 1 : 0); n <= last; ++n)
-                    mbar_wait_drain(&band_full[n % NB], (n / NB) & 1, p.timeout_ns);
+                    mbar_wait_drain(&band_full[n % NB], (n / NB) & 1);
         }
     } else if (warp == MMA_WARP || warp == MMA_WARP_B) {
         // ------------------------------------------------------------ MMA issuers
@@ -325,12 +347,12 @@ __global__ void __launch_bounds__(384, 1)
                 if (!is_b) IRA_TRACE(p, 23, n);
                 tc_fence_after();
                 const int st = n % NST, bb = n & 1;
-                // P^T / dS^T of query columns [32 w, 32 w + 32) sit, packed, at the
+                // P^T / dS^T of query columns [16 w, 16 w + 16) sit, packed, at the
                 // start of warpgroup w's own S / dP columns
                 const uint32_t cs = c_base(st);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {
-                    const uint32_t a_off = HALF * (kk >> 1) + 8 * (kk & 1);
+                    const uint32_t a_off = COLS * kk;
                     mma_ts(tmem + prod_col, tmem + col_of(bb) + a_off, sdesc_sw128(cs + kk * 2048, QTILE, 1024),
                            IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -339,19 +361,19 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (ok) mma_commit(acc_full);
             mma_commit(drain);
-            mbar_wait_drain(drain, 0, p.timeout_ns);
+            mbar_wait_drain(drain, 0);
         }
     }
     } else {
-        setmaxnreg_inc<208>();
+        setmaxnreg_inc<L::REG_EW>();
         // ------------------------------------------------------------ elementwise warpgroups
-        const int w = warp >> 2;       // this warpgroup takes query columns [32 w, 32 w + 32) of every step
+        const int w = warp >> 2;       // this warpgroup takes query columns [16 w, 16 w + 16) of every step
         const int wq = warp & 3;
         const int r = wq * 32 + lane;  // key row (TMEM lane)
         const int j = j0 + r;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
         const int tid = threadIdx.x & 127;
-        const int cw = HALF * w;       // first query column of this warpgroup
+        const int cw = COLS * w;       // first query column of this warpgroup
 
         bool ok = true;
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
@@ -367,64 +389,66 @@ __global__ void __launch_bounds__(384, 1)
                 ok = false;
                 break;
             }
-            if (tid == 0) IRA_TRACE(p, 25 + 3 * w, n);
+            if (tid == 0 && w < 2) IRA_TRACE(p, 25 + 3 * w, n);
             tc_fence_after();
-            uint32_t sv[HALF], dp[HALF];
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + cw, sv);
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + cw, dp);
+            uint32_t sv[COLS], dp[COLS];
+            tmem_ld16(tmem + lane_base + L::s_col(bb) + cw, sv);
+            tmem_ld16(tmem + lane_base + L::dp_col(bb) + cw, dp);
 
             // Band reads. Column c = cw + cl reads element (m + 127 - r) of shared band row
             // dm + c, where m = (dm + c) mod 8 repeats every 8 columns (cw is a multiple
             // of 8): eight per-step shared addresses plus compile-time offsets cover them all.
             const int dm = (delta - 127) & 7;
             const uint32_t band_s = smem_u32(smem + L::BAND_OFF + buf * BAND_BYTES + (dm + cw) * BAND_PITCH);
-            uint32_t baddr[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) baddr[u] = band_s + u * BAND_PITCH + 2 * (((dm + u) & 7) + 127 - r);
             const uint32_t info_s = smem_u32(smem + L::INFO_OFF + buf * int(sizeof(StepInfo)));
-            const bool full = lds_s32(info_s + offsetof(StepInfo, full)) != 0;
+            const bool info_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, info_s - smem_base, sizeof(StepInfo), L::TOTAL);
+            const bool full = info_ok && lds_s32(info_s + offsetof(StepInfo, full)) != 0;
             // dprofiles[b, h, i0 + c, delta + c - r] for column c = cw + cl: the address of
             // column cl is dbase + cl (R + 1) floats
-            char* const dbase = reinterpret_cast<char*>(
-                p.dprofiles + ((size_t(b) * p.Hq + h) * p.S + i0 + cw) * size_t(p.R) + (delta + cw - r));
+            const long long dp_at0 = ((long long)(b * p.Hq + h) * p.S + i0 + cw) * p.R + (delta + cw - r);
+            [[maybe_unused]] const long long dprof_n = n_rows * p.R;
+            char* const dbase = reinterpret_cast<char*>(p.dprofiles + dp_at0);
             const uint32_t dstride4 = 4u * uint32_t(p.R + 1);
             // d = delta + c - r < R  <=>  c < R - delta + r (no limit when the whole step is inside R)
             const bool inside = delta + BQ - 1 < p.R;
             const int cl_lim = (inside ? BQ : p.R - delta + r) - cw;
             tmem_wait_ld();
-            if (tid == 0) IRA_TRACE(p, 31, n);
-            uint32_t pk[HALF / 2], dk[HALF / 2];
+            if (tid == 0 && w == 0) IRA_TRACE(p, 31, n);
+            uint32_t pk[COLS / 2], dk[COLS / 2];
             // USED: the step reads profile entries; PLAIN: every (key, query) pair of the
             // step is allowed and inside R, so there is no mask and no store predicate
             auto math = [&](auto used_c, auto plain_c) {
                 constexpr bool USED = decltype(used_c)::value, PLAIN = decltype(plain_c)::value;
 #pragma unroll
-                for (int c16 = 0; c16 < HALF / 16; ++c16) {
-                    // loads of this 16-column chunk, issued together
-                    float nl_c[16], nv_c[16], bias_c[16];
-                    int lo_c[16], hi_c[16];
+                for (int c4 = 0; c4 < COLS / 4; ++c4) {
+                    // loads of this 4-column chunk: 128-bit broadcast reads of the column info
+                    const int c = cw + 4 * c4;
+                    const float4 l4 = info_ok ? lds_f32x4(info_s + offsetof(StepInfo, nlse2) + 4 * c)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 v4 = info_ok ? lds_f32x4(info_s + offsetof(StepInfo, ndv) + 4 * c)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float nl_c[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float nv_c[4] = {v4.x, v4.y, v4.z, v4.w};
+                    int lo_c[4] = {0, 0, 0, 0}, hi_c[4] = {0, 0, 0, 0};
+                    if (!PLAIN && info_ok) {
+                        const int4 a4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c);
+                        const int4 b4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c + 16);
+                        lo_c[0] = a4.x; hi_c[0] = a4.y; lo_c[1] = a4.z; hi_c[1] = a4.w;
+                        lo_c[2] = b4.x; hi_c[2] = b4.y; lo_c[3] = b4.z; hi_c[3] = b4.w;
+                    }
+                    float bias_c[4];
 #pragma unroll
-                    for (int u4 = 0; u4 < 4; ++u4) {  // 128-bit broadcast reads of four columns
-                        const int c = cw + 16 * c16 + 4 * u4;
-                        const float4 l4 = lds_f32x4(info_s + offsetof(StepInfo, nlse2) + 4 * c);
-                        const float4 v4 = lds_f32x4(info_s + offsetof(StepInfo, ndv) + 4 * c);
-                        nl_c[4 * u4 + 0] = l4.x; nl_c[4 * u4 + 1] = l4.y; nl_c[4 * u4 + 2] = l4.z; nl_c[4 * u4 + 3] = l4.w;
-                        nv_c[4 * u4 + 0] = v4.x; nv_c[4 * u4 + 1] = v4.y; nv_c[4 * u4 + 2] = v4.z; nv_c[4 * u4 + 3] = v4.w;
-                        if (!PLAIN) {
-                            const int4 a4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c);
-                            const int4 b4 = lds_s32x4(info_s + offsetof(StepInfo, rb) + 8 * c + 16);
-                            lo_c[4 * u4 + 0] = a4.x; hi_c[4 * u4 + 0] = a4.y; lo_c[4 * u4 + 1] = a4.z; hi_c[4 * u4 + 1] = a4.w;
-                            lo_c[4 * u4 + 2] = b4.x; hi_c[4 * u4 + 2] = b4.y; lo_c[4 * u4 + 3] = b4.z; hi_c[4 * u4 + 3] = b4.w;
-                        }
+                    for (int u = 0; u < 4; ++u) {
+                        const int cl = 4 * c4 + u;
+                        const uint32_t ba = band_s + (cl & 7) * BAND_PITCH + 2 * (((dm + cl) & 7) + 127 - r) +
+                                            BAND_PITCH * 8 * (cl >> 3);
+                        bias_c[u] = USED && IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, ba - smem_base, 2, L::TOTAL)
+                                        ? __uint_as_float(lds_u16(ba) << 16)
+                                        : 0.f;
                     }
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int cl = 16 * c16 + u;
-                        bias_c[u] = USED ? __uint_as_float(lds_u16(baddr[cl & 7] + BAND_PITCH * 8 * (cl >> 3)) << 16) : 0.f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const int cl = 16 * c16 + u;
+                    for (int u = 0; u < 4; u += 2) {
+                        const int cl = 4 * c4 + u;
                         // log2-domain logit, probability, dS = P (dP - Dv), two columns at a time
                         float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[cl]), __uint_as_float(sv[cl + 1])), sl2,
                                               make_float2(nl_c[u], nl_c[u + 1]));
@@ -442,8 +466,12 @@ __global__ void __launch_bounds__(384, 1)
                                            make_float2(nv_c[u], nv_c[u + 1])));
                         float* const a0 = reinterpret_cast<float*>(dbase + size_t(uint32_t(cl) * dstride4));
                         float* const a1 = reinterpret_cast<float*>(dbase + size_t(uint32_t(cl + 1) * dstride4));
-                        if (PLAIN || ok0) __stcs(a0, ds.x);
-                        if (PLAIN || ok1) __stcs(a1, ds.y);
+                        if ((PLAIN || ok0) &&
+                            IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, dp_at0 + (long long)cl * (p.R + 1), 1, dprof_n))
+                            __stcs(a0, ds.x);
+                        if ((PLAIN || ok1) && IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal,
+                                                            dp_at0 + (long long)(cl + 1) * (p.R + 1), 1, dprof_n))
+                            __stcs(a1, ds.y);
                         pk[cl >> 1] = pack_bf16x2(pr.x, pr.y);
                         dk[cl >> 1] = pack_bf16x2(ds.x, ds.y);
                     }
@@ -456,9 +484,9 @@ __global__ void __launch_bounds__(384, 1)
             } else {
                 if (full && inside) math(F_{}, T_{}); else math(F_{}, F_{});
             }
-            if (tid == 0) IRA_TRACE(p, 32, n);
-            tmem_st16(tmem + lane_base + L::s_col(bb) + cw, pk);
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + cw, dk);
+            if (tid == 0 && w == 0) IRA_TRACE(p, 32, n);
+            tmem_st8(tmem + lane_base + L::s_col(bb) + cw, pk);
+            tmem_st8(tmem + lane_base + L::dp_col(bb) + cw, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -466,20 +494,23 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive(&p_full[bb]);
                 mbar_arrive(&band_empty[buf]);
             }
-            if (tid == 0) IRA_TRACE(p, 26 + 3 * w, n);
+            if (tid == 0 && w < 2) IRA_TRACE(p, 26 + 3 * w, n);
         }
 
-        // ---- epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV ----
+        // ---- epilogue: warpgroups 0 and 1 write dK (scaled), 2 and 3 dV, half of the
+        // columns each ----
         if (ok && n_steps > 0) {
             ok = warp_wait(acc_full, 0, ctl, p.err, kErrDkdvAcc, p.timeout_ns);
             tc_fence_after();
         }
         if (ok) {
             const bool row_in = j < p.Skv;
-            float* dst = (w == 0 ? p.dk : p.dv) + (b * p.kv_sb + j * p.kv_ss + g * p.kv_sh);
-            float* const base = (w == 0 ? p.dk : p.dv) + (b * p.kv_sb + g * p.kv_sh);
-            const float mul = (w == 0) ? p.scale : 1.f;
-            const uint32_t col = (w == 0) ? L::DK_COL : L::DV_COL;
+            const bool is_dv = w >= 2;
+            const int c0 = (w & 1) * (D / 2);  // first of this warpgroup's D / 2 columns
+            float* dst = (is_dv ? p.dv : p.dk) + (b * p.kv_sb + j * p.kv_ss + g * p.kv_sh);
+            float* const base = (is_dv ? p.dv : p.dk) + (b * p.kv_sb + g * p.kv_sh);
+            const float mul = is_dv ? 1.f : p.scale;
+            const uint32_t col = (is_dv ? L::DV_COL : L::DK_COL) + c0;
             if (n_steps > 0) {
                 // 32 x 32 chunks go out through shared memory (the key / query tiles, idle once
                 // every MMA has completed), 144-byte pitch per row: each lane writes its row,
@@ -488,27 +519,39 @@ __global__ void __launch_bounds__(384, 1)
                 float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * 36;
                 const int sr = lane >> 3, sc = 4 * (lane & 7);
 #pragma unroll 1
-                for (int c4 = 0; c4 < D / 32; ++c4) {
+                for (int c4 = 0; c4 < D / 64; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + col + 32 * c4, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<float4*>(stage + lane * 36 + 4 * q) =
-                            make_float4(__uint_as_float(o[4 * q]) * mul, __uint_as_float(o[4 * q + 1]) * mul,
-                                        __uint_as_float(o[4 * q + 2]) * mul, __uint_as_float(o[4 * q + 3]) * mul);
+                        if (IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, smem_u32(stage + lane * 36 + 4 * q) - smem_base, 16,
+                                          L::TOTAL))
+                            *reinterpret_cast<float4*>(stage + lane * 36 + 4 * q) =
+                                make_float4(__uint_as_float(o[4 * q]) * mul, __uint_as_float(o[4 * q + 1]) * mul,
+                                            __uint_as_float(o[4 * q + 2]) * mul, __uint_as_float(o[4 * q + 3]) * mul);
                     __syncwarp();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int rr = 4 * k + sr;          // row of this warp
                         const int jr = j0 + 32 * wq + rr;   // its key
-                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * 36 + sc);
-                        if (jr < p.Skv) *reinterpret_cast<float4*>(base + jr * p.kv_ss + 32 * c4 + sc) = v;
+                        const bool st_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDkdvSmem, smem_u32(stage + rr * 36 + sc) - smem_base,
+                                                         16, L::TOTAL);
+                        const float4 v = st_ok ? *reinterpret_cast<const float4*>(stage + rr * 36 + sc)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                        [[maybe_unused]] const long long at =
+                            b * p.kv_sb + g * p.kv_sh + (long long)jr * p.kv_ss + c0 + 32 * c4 + sc;
+                        if (jr < p.Skv &&
+                            IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal, at, 4, (long long)p.B * p.Skv * p.Hkv * D))
+                            *reinterpret_cast<float4*>(base + jr * p.kv_ss + c0 + 32 * c4 + sc) = v;
                     }
                     __syncwarp();
                 }
-            } else if (row_in) {
-                for (int e = 0; e < D; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (row_in && IRA_IN_BOUNDS(p.err, kErrBoundsDkdvGlobal,
+                                               b * p.kv_sb + (long long)j * p.kv_ss + g * p.kv_sh + c0, D / 2,
+                                               (long long)p.B * p.Skv * p.Hkv * D)) {
+                for (int e = c0; e < c0 + D / 2; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
     }
@@ -531,7 +574,7 @@ cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUten
     const int nkt = (p.Skv + BK - 1) / BK;
     const long long grid = (long long)nkt * p.B * p.Hkv;
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, tm_band, p, nkt);
+    kern<<<dim3(unsigned(grid)), dim3(32 * L::NWARPS), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, tm_band, p, nkt);
     return cudaGetLastError();
 }
 
@@ -544,8 +587,9 @@ namespace dqk {
 
 constexpr int BM = 128;               // query rows per CTA (TMEM lanes)
 constexpr int BN = 64;                // keys per step
-constexpr int HALF = BN / 2;          // key columns per elementwise warpgroup
-constexpr int BAND_CHUNKS = 5;        // 40 bf16 per row window (32 columns + misalignment)
+constexpr int NWG = 4;                // elementwise warpgroups
+constexpr int COLS = BN / NWG;        // key columns per elementwise warpgroup
+constexpr int BAND_CHUNKS = 3;        // 24 bf16 per row window (16 columns + misalignment)
 constexpr int BAND_UNITS = BAND_CHUNKS * BM + 2 * (BM / 8);
 constexpr int BAND_BYTES = BAND_UNITS * 16;
 constexpr int QTILE = BM * 128;       // [128 x 64 bf16]
@@ -554,6 +598,9 @@ constexpr int NSB = 3;                // S / dP buffers in TMEM: the MMAs run tw
 constexpr int NSK = 4;                // K stages: K(n) is read by S(n) and, two steps later, by dQ(n)
 constexpr int NSV = 2;                // V stages: V(n) is read by dP(n) only
 
+// Row r's window starts at 16-byte unit 3 r + 2 floor(r / 8) of its buffer; with the
+// row's misalignment (r + 1) mod 8 the column-wise 32-bit reads of a warp hit 32
+// distinct banks.
 __host__ __device__ constexpr int band_unit(int r) { return BAND_CHUNKS * r + 2 * (r >> 3); }
 
 template <int D>
@@ -564,7 +611,11 @@ struct Layout {
     static constexpr int K_OFF = DO_OFF + KB * QTILE;          // NSK stages
     static constexpr int V_OFF = K_OFF + NSK * KB * KTILE;     // NSV stages
     static constexpr int BAND_OFF = V_OFF + NSV * KB * KTILE;  // [warpgroup][step parity]
-    static constexpr int BAR_OFF = BAND_OFF + 4 * BAND_BYTES;
+    // fused L2Clip backward: row sums [lane quarter][warpgroup][lane] float2, then column
+    // sums [warpgroup][lane quarter][column] floats
+    static constexpr int XCH_OFF = BAND_OFF + NWG * 2 * BAND_BYTES;
+    static constexpr int XCH_BYTES = 4 * NWG * 32 * 8 + NWG * 4 * 32 * 4;
+    static constexpr int BAR_OFF = XCH_OFF + XCH_BYTES;
     // q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[NSB], p_full[NSB],
     // acc_full, drain
     static constexpr int NBARS = 3 + 2 * NSK + 2 * NSV + 2 * NSB;
@@ -575,16 +626,29 @@ struct Layout {
     static constexpr uint32_t s_col(int bb) { return uint32_t(D + 128 * bb); }
     static constexpr uint32_t dp_col(int bb) { return uint32_t(D + 128 * bb + 64); }
     static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int NWARPS = 4 * NWG + 4;
+    // registers per thread at launch, and after the split: control warpgroup / elementwise
+    static constexpr int REG_LAUNCH = 96, REG_CTRL = 56, REG_EW = 104;
+    static_assert(128 * REG_CTRL + 128 * NWG * REG_EW <= 32 * NWARPS * REG_LAUNCH, "register split");
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    // the epilogue stages the D / NWG dQ columns of each warp's 32 rows through the K
+    // and V rings (contiguous, idle by then), 4 floats of padding per row
+    static constexpr int DC = D / NWG;
+    static constexpr int STAGE_PITCH = DC + 4;
+    static_assert(4 * NWG * 32 * STAGE_PITCH * 4 <= (NSK + NSV) * KB * KTILE, "epilogue staging");
 };
 
-template <int D>
-__global__ void __launch_bounds__(384, 1)
+// CLIP: the L2Clip backward of q is fused into the epilogue (dq of the clipped q becomes
+// the gradient of the unclipped q, plus this CTA's parts of dscale and dtau).
+template <int D, bool CLIP>
+__global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const AttnParams p, const int num_qtiles) {
     using L = Layout<D>;
     constexpr int KB = L::KB;
-    constexpr int TMA_WARP = 8, MMA_WARP = 9, V_WARP = 10, MMA_WARP_B = 11;
+    constexpr int CTRL = 4 * NWG;
+    constexpr int TMA_WARP = CTRL, MMA_WARP = CTRL + 1, V_WARP = CTRL + 2, MMA_WARP_B = CTRL + 3;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the __shared__ array, so the compiler keeps
     // knowing that every pointer derived from it addresses shared memory
@@ -612,10 +676,12 @@ __global__ void __launch_bounds__(384, 1)
     const int i0 = qt * BM;
     const int i0g = p.q_off + i0;
     const int t64 = (p.S + 63) / 64;
+    // buffer extents for the bounds-checking build (elements; shared memory in bytes)
+    [[maybe_unused]] const uint32_t smem_base = smem_u32(smem);
+    [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        // a K / V stage is free, and S / dP of a step ready, once both MMA issuers committed
         // a K stage is free once S (issuer A) and dQ (issuer B) of its step completed,
         // a V stage once dP (issuer B) did
         for (int u = 0; u < NSK; ++u) {
@@ -627,15 +693,17 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&v_empty[u], 1);
         }
         for (int u = 0; u < NSB; ++u) {
-            mbar_init(&s_full[u], 2);
-            mbar_init(&p_full[u], 8);
+            mbar_init(&s_full[u], 2);           // S (issuer A) and dP (issuer B)
+            mbar_init(&p_full[u], 4 * NWG);     // every elementwise warp
         }
         mbar_init(acc_full, 1);
         mbar_init(drain, 2);
         ctl->abort = 0;
         const TileBounds* tb = p.tile_bounds + size_t(b) * t64 + 2 * qt;
-        int min_lo = tb[0].min_lo, max_hi = tb[0].max_hi, ne = tb[0].n_nonempty;
-        if (2 * qt + 1 < t64) {
+        const bool tb_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, size_t(b) * t64 + 2 * qt,
+                                         (2 * qt + 1 < t64) ? 2 : 1, (long long)p.B * t64);
+        int min_lo = tb_ok ? tb[0].min_lo : 0, max_hi = tb_ok ? tb[0].max_hi : -1, ne = tb_ok ? tb[0].n_nonempty : 0;
+        if (tb_ok && 2 * qt + 1 < t64) {
             min_lo = min(min_lo, tb[1].min_lo);
             max_hi = max(max_hi, tb[1].max_hi);
             ne += tb[1].n_nonempty;
@@ -668,11 +736,11 @@ __global__ void __launch_bounds__(384, 1)
     auto v_smem = [&](int n, int kb) { return smem + L::V_OFF + ((n % NSV) * KB + kb) * KTILE; };
     auto key0 = [&](int n) { return i0g + BN - (t_begin + n) * BN; };
 
-    // Launched with 384 x 168 registers; warpgroup 2 (producer, two MMA issuers, an idle
-    // warp) gives part of its share to the two elementwise warpgroups
-    // (128 x 80 + 256 x 208 <= 384 x 168). Each change sits at the top of its branch.
-    if (warp >= 8) {
-        setmaxnreg_dec<80>();
+    // Launched with REG_LAUNCH registers per thread; the control warpgroup (producers,
+    // two MMA issuers) gives part of its share to the elementwise warpgroups (checked
+    // against the launch total above). Each change sits at the top of its branch.
+    if (warp >= CTRL) {
+        setmaxnreg_dec<L::REG_CTRL>();
     if (warp == TMA_WARP || warp == V_WARP) {
         // ------------------------------------------------------------ tile producers:
         // Q and dO once plus the K ring (TMA_WARP), the V ring (V_WARP)
@@ -707,9 +775,9 @@ __global__ void __launch_bounds__(384, 1)
                 if (!is_v) IRA_TRACE(p, 41, n);
                 last = n;
             }
-            if (!is_v) mbar_wait_drain(q_full, 0, p.timeout_ns);
+            if (!is_v) mbar_wait_drain(q_full, 0);
             for (int n = (last >= ns ? last - ns + 1 : 0); n <= last; ++n)
-                mbar_wait_drain(&full[n % ns], (n / ns) & 1, p.timeout_ns);
+                mbar_wait_drain(&full[n % ns], (n / ns) & 1);
         }
     } else if (warp == MMA_WARP || warp == MMA_WARP_B) {
         // ------------------------------------------------------------ MMA issuers
@@ -775,9 +843,9 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t ks = smem_u32(k_smem(n, 0));
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    // dS of key columns [32 w, 32 w + 32) sits, packed, at the start of
-                    // warpgroup w's own dP columns
-                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + HALF * (kk >> 1) + 8 * (kk & 1),
+                    // dS of key columns [16 w, 16 w + 16) sits, packed, at the start of
+                    // warpgroup w's own 16 dP columns
+                    mma_ts(tmem + L::DQ_COL, tmem + L::dp_col(bb) + COLS * kk,
                            sdesc_sw128(ks + kk * 2048, KTILE, 1024), IDESC_DQ, (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&k_empty[n % NSK]);
@@ -785,51 +853,54 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (ok && is_b) mma_commit(acc_full);
             mma_commit(drain);
-            mbar_wait_drain(drain, 0, p.timeout_ns);
+            mbar_wait_drain(drain, 0);
         }
     }
     } else {
-        setmaxnreg_inc<208>();
-        const int w = warp >> 2;       // this warpgroup takes key columns [32 w, 32 w + 32) of every step
+        setmaxnreg_inc<L::REG_EW>();
+        const int w = warp >> 2;       // this warpgroup takes key columns [16 w, 16 w + 16) of every step
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t lane_base = uint32_t(wq * 32) << 16;
-        const int cw = HALF * w;
+        const int cw = COLS * w;
         const int i = i0 + r;
-        const bool row_in = i < p.S;
+        const size_t trow = (size_t(b) * p.Hq + h) * p.S + i;
+        const bool row_in = i < p.S &&
+                            IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, size_t(b) * p.S + i, 1, (long long)p.B * p.S) &&
+                            IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, trow, 1, n_rows);
         const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
         const bool empty = rb.x > rb.y;
-        const size_t trow = (size_t(b) * p.Hq + h) * p.S + i;
         const float lse2 = row_in ? p.lse2t[trow] : 0.f;
         const float dvr = row_in ? p.dvt[trow] : 0.f;
 
         // This thread's profile window for its columns, double buffered by step parity:
-        // column c = cw + cl of step n has distance delta(n) + r - c; the 32 columns'
+        // column c = cw + cl of step n has distance delta(n) + r - c; the 16 columns'
         // window starts (r + 1) mod 8 elements past a 16-byte boundary.
         const int unit = band_unit(r);
-        auto band_saddr = [&](int buf) {
-            return smem_u32(smem + L::BAND_OFF + (2 * w + buf) * BAND_BYTES) + uint32_t(unit) * 16u;
-        };
+        uint8_t* const band_wg = smem + L::BAND_OFF + w * 2 * BAND_BYTES;
         const int m_r = (r + 1) & 7;
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
-        const uint16_t* prof_row =
-            (p.R > 0 && row_in && !empty) ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) : nullptr;
+        const size_t prof_at = trow * size_t(p.R);
+        const uint16_t* prof_row = (p.R > 0 && row_in && !empty) ? p.profiles + prof_at : nullptr;
+        [[maybe_unused]] const long long prof_n = n_rows * p.R;
         // step n has distance offset delta = i0g - key0(n) = 64 (t_begin + n) - 64
         auto delta_of = [&](int n) { return BN * (t_begin + n) - BN; };
-        // the warp's smallest distance in this warpgroup's columns is delta + 32 wq - cw - 31
-        auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - cw - (HALF - 1) < p.R; };
+        // the warp's smallest distance in this warpgroup's columns is delta + 32 wq - cw - 15
+        auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - cw - (COLS - 1) < p.R; };
         // one cp.async group per call, also when nothing is copied
         auto issue_band = [&](int n) {
             if (n < n_steps && band_needed(n)) {
-                const int x0 = delta_of(n) + r - cw - (HALF - 1) - m_r;
-                const uint32_t dst = band_saddr(n & 1);
+                const int x0 = delta_of(n) + r - cw - (COLS - 1) - m_r;
+                const uint32_t dst = smem_u32(band_wg + (n & 1) * BAND_BYTES) + uint32_t(unit) * 16u;
 #pragma unroll
                 for (int q = 0; q < BAND_CHUNKS; ++q) {
                     const int d0 = x0 + 8 * q;
                     const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
                     const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                    cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                    if (IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, dst + 16u * q - smem_base, 16, L::TOTAL) &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, inb ? prof_at + d0 : 0, inb ? 8 : 0, prof_n))
+                        cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
                 }
             }
             cp_async_commit();
@@ -845,37 +916,38 @@ __global__ void __launch_bounds__(384, 1)
         for (int n = 0; n < n_steps; ++n) {
             const int bb = n % NSB;
             const int jk = key0(n) + cw;  // key of this warpgroup's first column
-            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + HALF - 1);
+            const bool my_full = empty || (rb.x <= jk && rb.y >= jk + COLS - 1);
             const bool need_mask = !__all_sync(0xffffffffu, my_full);
             const bool use_band = band_needed(n);
             if (!warp_wait(&s_full[bb], (n / NSB) & 1, ctl, p.err, kErrDqS, p.timeout_ns)) {
                 ok = false;
                 break;
             }
-            if (wq == 0 && lane == 0) IRA_TRACE(p, 45 + 2 * w, n);
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 45 + 2 * (w & 1), n);
             tc_fence_after();
-            uint32_t sv[HALF], dp[HALF];
-            tmem_ld32(tmem + lane_base + L::s_col(bb) + cw, sv);
-            tmem_ld32(tmem + lane_base + L::dp_col(bb) + cw, dp);
-            uint32_t wv[17];
+            uint32_t sv[COLS], dp[COLS];
+            tmem_ld16(tmem + lane_base + L::s_col(bb) + cw, sv);
+            tmem_ld16(tmem + lane_base + L::dp_col(bb) + cw, dp);
+            uint32_t wv[COLS / 2 + 1];
             if (use_band) {
                 cp_async_wait_group<1>();  // this step's window (the next step's may fly)
-                const uint32_t* words =
-                    reinterpret_cast<const uint32_t*>(smem + L::BAND_OFF + (2 * w + (n & 1)) * BAND_BYTES + unit * 16) + g_r;
+                const uint32_t* words = reinterpret_cast<const uint32_t*>(band_wg + (n & 1) * BAND_BYTES + unit * 16) + g_r;
+                const bool w_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, smem_u32(words) - smem_base,
+                                                4 * (COLS / 2 + 1), L::TOTAL);
 #pragma unroll
-                for (int q = 0; q < 17; ++q) wv[q] = words[q];
+                for (int q = 0; q < COLS / 2 + 1; ++q) wv[q] = w_ok ? words[q] : 0u;
             }
             // this step's window is in registers: fetch the one of step n + 2 into its buffer
             issue_band(n + 2);
             tmem_wait_ld();
             const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
-            uint32_t dk[HALF / 2];
+            uint32_t dk[COLS / 2];
 #pragma unroll
-            for (int pp = 0; pp < HALF / 2; ++pp) {
+            for (int pp = 0; pp < COLS / 2; ++pp) {
                 const int c = 2 * pp;
                 float2 t = nl2;
                 if (use_band) {
-                    const uint32_t v = funnel_r(wv[15 - pp], wv[16 - pp], fshift);
+                    const uint32_t v = funnel_r(wv[COLS / 2 - 1 - pp], wv[COLS / 2 - pp], fshift);
                     t = __ffma2_rn(make_float2(bf16hi_to_f32(v), bf16lo_to_f32(v)), l2e, nl2);
                 }
                 const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
@@ -888,58 +960,180 @@ __global__ void __launch_bounds__(384, 1)
                     __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv2));
                 dk[pp] = pack_bf16x2(ds.x, ds.y);
             }
-            tmem_st16(tmem + lane_base + L::dp_col(bb) + cw, dk);
+            tmem_st8(tmem + lane_base + L::dp_col(bb) + cw, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[bb]);
-            if (wq == 0 && lane == 0) IRA_TRACE(p, 46 + 2 * w, n);
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 46 + 2 * (w & 1), n);
         }
         cp_async_wait_all();
 
-        // ---- epilogue: each warpgroup writes half of the dQ columns ----
+        // Fused L2Clip backward (CLIP). dy = dq of the clipped q; per row (b, i, h):
+        //   z = x * scale, n = |z|, c = min(1, thr / n);
+        //   dz = tau c (dy - ((z . dy) / n^2) z) when n > thr, else tau dy;
+        //   dx = dz * scale (written where dq goes), dtau part c (z . dy), dscale part dz * x.
+        // Each warpgroup holds a quarter of the columns: the row sums z . z and z . dy go
+        // through shared memory among the four warps of a lane quarter (barrier 1 + wq), the
+        // column sums of dz * x over the CTA's rows among the four warps of a warpgroup
+        // (barrier 5 + w); both in a fixed order. Every warp takes both barriers, also after
+        // a failed wait; only the stores depend on it.
+        auto clip_epilogue = [&](bool ok_out) {
+            constexpr int DC = L::DC, STAGE_PITCH = L::STAGE_PITCH;
+            const int col = w * DC;
+            float dy[DC];
+            if (ok_out && n_steps > 0) {
+                uint32_t o[DC];
+                if constexpr (DC == 32) {
+                    tmem_ld32(tmem + lane_base + L::DQ_COL + col, o);
+                } else {
+                    tmem_ld16(tmem + lane_base + L::DQ_COL + col, o);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < DC; ++e) dy[e] = empty ? 0.f : __uint_as_float(o[e]) * p.scale;
+            } else {
+#pragma unroll
+                for (int e = 0; e < DC; ++e) dy[e] = 0.f;
+            }
+            float xv[DC];
+            const size_t xrow = ((size_t(b) * p.S + i) * p.Hq + h) * D + col;
+#pragma unroll
+            for (int e8 = 0; e8 < DC / 8; ++e8) {
+                const uint4 u = row_in ? *reinterpret_cast<const uint4*>(p.q_raw + xrow + 8 * e8) : make_uint4(0, 0, 0, 0);
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    xv[8 * e8 + 2 * e] = bf16lo_to_f32(wv[e]);
+                    xv[8 * e8 + 2 * e + 1] = bf16hi_to_f32(wv[e]);
+                }
+            }
+            const float* const scl = p.clip_scale ? p.clip_scale + size_t(h) * D + col : nullptr;
+            auto scv = [&](int e) { return scl ? scl[e] : 1.f; };
+            float zz = 0.f, zd = 0.f;
+#pragma unroll
+            for (int e = 0; e < DC; ++e) {
+                const float z = xv[e] * scv(e);
+                zz = fmaf(z, z, zz);
+                zd = fmaf(z, dy[e], zd);
+            }
+            float2* const xrows = reinterpret_cast<float2*>(smem + L::XCH_OFF);
+            float* const csum = reinterpret_cast<float*>(smem + L::XCH_OFF + 4 * NWG * 32 * 8);
+            xrows[(wq * NWG + w) * 32 + lane] = make_float2(zz, zd);
+            named_bar_sync(1 + wq, 32 * NWG);
+            float zz_t = 0.f, zd_t = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < NWG; ++w2) {
+                const float2 v = xrows[(wq * NWG + w2) * 32 + lane];
+                zz_t += v.x;
+                zd_t += v.y;
+            }
+            const float nrm = sqrtf(zz_t);
+            const bool clipped = nrm > p.clip_thr;
+            const float c = clipped ? p.clip_thr / nrm : 1.f;
+            const float tau = (p.clip_tau && row_in) ? p.clip_tau[size_t(b) * p.S + i] : 1.f;
+            const float k2 = clipped ? zd_t / zz_t : 0.f;
+            if (ok_out && w == 0 && row_in) p.dtau_part[(size_t(b) * p.S + i) * p.Hq + h] = c * zd_t;
+            // dz * x of this warp's rows, summed down the rows (a lane per column), then over
+            // the four warps of the warpgroup
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * STAGE_PITCH;
+#pragma unroll
+            for (int e = 0; e < DC; ++e) {  // dy becomes dx
+                const float dz = tau * c * (dy[e] - k2 * (xv[e] * scv(e)));
+                dy[e] = dz * scv(e);
+                stage[lane * STAGE_PITCH + e] = dz * xv[e];
+            }
+            __syncwarp();
+            if (lane < DC) {
+                float a = 0.f;
+                for (int rr = 0; rr < 32; ++rr) a += stage[rr * STAGE_PITCH + lane];
+                csum[(w * 4 + wq) * 32 + lane] = a;
+            }
+            named_bar_sync(5 + w, 128);
+            if (ok_out && wq == 0 && lane < DC) {
+                const float a = (csum[(w * 4 + 0) * 32 + lane] + csum[(w * 4 + 1) * 32 + lane]) +
+                                (csum[(w * 4 + 2) * 32 + lane] + csum[(w * 4 + 3) * 32 + lane]);
+                p.dscale_part[((size_t(b) * num_qtiles + qt) * p.Hq + h) * D + col + lane] = a;
+            }
+            __syncwarp();
+            // dx leaves through the same staging rows: each lane writes its row, then DC / 4
+            // lanes store the row's DC contiguous floats
+#pragma unroll
+            for (int e = 0; e < DC; e += 4)
+                *reinterpret_cast<float4*>(stage + lane * STAGE_PITCH + e) = make_float4(dy[e], dy[e + 1], dy[e + 2], dy[e + 3]);
+            __syncwarp();
+            constexpr int LPR = DC / 4;       // lanes per row
+            constexpr int RPI = 32 / LPR;     // rows per store instruction
+            const int sr = lane / LPR, sc = 4 * (lane % LPR);
+            float* const base = p.dq + (b * p.row_sb + h * p.row_sh);
+            if (ok_out) {
+#pragma unroll
+                for (int k = 0; k < 32 / RPI; ++k) {
+                    const int rr = RPI * k + sr;        // row of this warp
+                    const int ir = i0 + 32 * wq + rr;   // its query row
+                    const float4 v = *reinterpret_cast<const float4*>(stage + rr * STAGE_PITCH + sc);
+                    if (ir < p.S) *reinterpret_cast<float4*>(base + ir * p.row_ss + col + sc) = v;
+                }
+            }
+        };
+
+        // ---- epilogue: each warpgroup writes a quarter of the dQ columns ----
         if (ok && n_steps > 0) {
             ok = warp_wait(acc_full, 0, ctl, p.err, kErrDqAcc, p.timeout_ns);
             tc_fence_after();
         }
-        if (ok) {
+        if constexpr (CLIP) {
+            clip_epilogue(ok);
+        } else if (ok) {
+            constexpr int DC = L::DC, STAGE_PITCH = L::STAGE_PITCH;  // dQ columns of this warpgroup
+            const int col = w * DC;
             float* dst = p.dq + (b * p.row_sb + i * p.row_ss + h * p.row_sh);
             float* const base = p.dq + (b * p.row_sb + h * p.row_sh);
-            constexpr int HALF = D / 2;
             if (n_steps > 0) {
-                // 32 x 32 chunks go out through shared memory (the K / V rings, idle once every
-                // MMA has completed), 144-byte pitch per row: each lane writes its row, then
-                // 8 lanes store 128 contiguous bytes of one row, four rows per store
+                // the rows leave through shared memory (the K / V rings, idle once every MMA
+                // has completed): each lane writes its row, then DC / 4 lanes store the row's
+                // DC contiguous floats
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * 36;
-                const int sr = lane >> 3, sc = 4 * (lane & 7);
-#pragma unroll 1
-                for (int c4 = 0; c4 < HALF / 32; ++c4) {
-                    const int col = w * HALF + 32 * c4;
-                    uint32_t o[32];
+                float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * STAGE_PITCH;
+                constexpr int LPR = DC / 4;       // lanes per row
+                constexpr int RPI = 32 / LPR;     // rows per store instruction
+                const int sr = lane / LPR, sc = 4 * (lane % LPR);
+                uint32_t o[DC];
+                if constexpr (DC == 32) {
                     tmem_ld32(tmem + lane_base + L::DQ_COL + col, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 v;
-                        v.x = empty ? 0.f : __uint_as_float(o[4 * q]) * p.scale;
-                        v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * p.scale;
-                        v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * p.scale;
-                        v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * p.scale;
-                        *reinterpret_cast<float4*>(stage + lane * 36 + 4 * q) = v;
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int rr = 4 * k + sr;          // row of this warp
-                        const int ir = i0 + 32 * wq + rr;   // its query row
-                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * 36 + sc);
-                        if (ir < p.S) *reinterpret_cast<float4*>(base + ir * p.row_ss + col + sc) = v;
-                    }
-                    __syncwarp();
+                } else {
+                    tmem_ld16(tmem + lane_base + L::DQ_COL + col, o);
                 }
-            } else if (row_in) {
-                for (int e = w * HALF; e < (w + 1) * HALF; e += 4)
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < DC / 4; ++q) {
+                    float4 v;
+                    v.x = empty ? 0.f : __uint_as_float(o[4 * q]) * p.scale;
+                    v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * p.scale;
+                    v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * p.scale;
+                    v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * p.scale;
+                    if (IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, smem_u32(stage + lane * STAGE_PITCH + 4 * q) - smem_base,
+                                      16, L::TOTAL))
+                        *reinterpret_cast<float4*>(stage + lane * STAGE_PITCH + 4 * q) = v;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 32 / RPI; ++k) {
+                    const int rr = RPI * k + sr;        // row of this warp
+                    const int ir = i0 + 32 * wq + rr;   // its query row
+                    const bool st_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem,
+                                                     smem_u32(stage + rr * STAGE_PITCH + sc) - smem_base, 16, L::TOTAL);
+                    const float4 v = st_ok ? *reinterpret_cast<const float4*>(stage + rr * STAGE_PITCH + sc)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    [[maybe_unused]] const long long at = b * p.row_sb + h * p.row_sh + (long long)ir * p.row_ss + col + sc;
+                    if (ir < p.S && IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, at, 4, n_rows * D))
+                        *reinterpret_cast<float4*>(base + ir * p.row_ss + col + sc) = v;
+                }
+            } else if (row_in && IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal,
+                                               b * p.row_sb + (long long)i * p.row_ss + h * p.row_sh + col, DC,
+                                               n_rows * D)) {
+                for (int e = col; e < col + DC; e += 4)
                     *reinterpret_cast<float4*>(dst + e) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
@@ -953,17 +1147,17 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int D>
+template <int D, bool CLIP>
 cudaError_t launch(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                    const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
     using L = Layout<D>;
-    auto kern = dq_kernel<D>;
+    auto kern = dq_kernel<D, CLIP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     const int nqt = (p.S + BM - 1) / BM;
     const long long grid = (long long)nqt * p.B * p.Hq;
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(384), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nqt);
+    kern<<<dim3(unsigned(grid)), dim3(32 * L::NWARPS), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_do, p, nqt);
     return cudaGetLastError();
 }
 
@@ -979,8 +1173,11 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& tm_q, const CUtensorMap& tm_k, co
 
 cudaError_t launch_bwd_dq(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           const CUtensorMap& tm_do, const AttnParams& p, cudaStream_t st) {
-    return p.D == 128 ? bwdk::dqk::launch<128>(tm_q, tm_k, tm_v, tm_do, p, st)
-                      : bwdk::dqk::launch<64>(tm_q, tm_k, tm_v, tm_do, p, st);
+    if (p.q_raw)
+        return p.D == 128 ? bwdk::dqk::launch<128, true>(tm_q, tm_k, tm_v, tm_do, p, st)
+                          : bwdk::dqk::launch<64, true>(tm_q, tm_k, tm_v, tm_do, p, st);
+    return p.D == 128 ? bwdk::dqk::launch<128, false>(tm_q, tm_k, tm_v, tm_do, p, st)
+                      : bwdk::dqk::launch<64, false>(tm_q, tm_k, tm_v, tm_do, p, st);
 }
 
 }  // namespace ira

@@ -29,7 +29,27 @@ enum ErrSite : int {
     kErrDkdvKV = 201, kErrDkdvQ, kErrDkdvS, kErrDkdvP, kErrDkdvAcc, kErrDkdvQFree,
     kErrDqQ = 301, kErrDqKV, kErrDqS, kErrDqP, kErrDqAcc, kErrDqKVFree,
     kErrSelftest = 901,
+    // bounds-checking builds only: an index outside its buffer (the access is skipped)
+    kErrBoundsFwdSmem = 951, kErrBoundsFwdGlobal, kErrBoundsDkdvSmem, kErrBoundsDkdvGlobal, kErrBoundsDqSmem,
+    kErrBoundsDqGlobal,
 };
+
+// Index checks of the bounds-checking build (-DINKLING_BOUNDS_CHECK): IRA_IN_BOUNDS(err,
+// code, off, bytes, size) is true when the access [off, off + bytes) lies inside a buffer
+// of `size` bytes (or elements, as long as all three agree); otherwise it records `code`
+// in the device error word (first one wins) and is false, and the caller skips the
+// access. Nothing traps. In ordinary builds it is the constant true.
+#ifdef INKLING_BOUNDS_CHECK
+__device__ __forceinline__ bool ira_in_bounds(int* err, int code, long long off, long long bytes, long long size) {
+    if (off >= 0 && bytes >= 0 && off + bytes <= size) return true;
+    if (err) atomicCAS(err, 0, code);
+    return false;
+}
+#define IRA_IN_BOUNDS(err, code, off, bytes, size) \
+    ::ira::ira_in_bounds((err), (code), (long long)(off), (long long)(bytes), (long long)(size))
+#else
+#define IRA_IN_BOUNDS(err, code, off, bytes, size) true
+#endif
 
 // Per-64-row query tile summary written by the bounds kernel.
 struct TileBounds {
@@ -109,6 +129,16 @@ struct AttnParams {
     float* dk;
     float* dv;
     float* dprofiles;
+    // L2Clip of q fused into the attention (q_clipped set: the forward clips each Q tile
+    // and stores it; q_raw set: the dQ kernel turns dq into the gradient of the unclipped
+    // q): z = q_raw * clip_scale[h, :], q = z * min(1, clip_thr / |z|) * clip_tau[b, i]
+    float clip_thr;
+    const float* clip_scale;   // [Hq, D] or null
+    const float* clip_tau;     // [B, S] or null
+    uint16_t* q_clipped;       // forward: clipped q [B, S, Hq, D] BF16 (written)
+    const uint16_t* q_raw;     // dQ: unclipped q [B, S, Hq, D] BF16
+    float* dscale_part;        // dQ: parts of dscale, [B * ceil(S / 128)][Hq][D]
+    float* dtau_part;          // dQ: parts of dtau, [B, S, Hq]
     // pipeline timeline of one CTA (only in builds with INKLING_TRACE; null otherwise)
     unsigned long long* trace;
     int trace_cta;

@@ -78,8 +78,8 @@ struct Layout {
     static constexpr int BAND_OFF = V_OFF + VSLOTS * SLOT_BYTES;
     static constexpr int BAR_OFF = BAND_OFF + NH * 2 * BAND_BYTES;
     // q_full, k_first[2], kv_ready[NKV], k_empty[KSLOTS], v_empty[VSLOTS], drain,
-    // s_full[NH][2], p_full[NH][2], o_done[NH], o_full[NH]
-    static constexpr int NBARS = 4 + NKV + KSLOTS + VSLOTS + 6 * NH;
+    // s_full[NH][2], p_full[NH][2], o_done[NH], o_full[NH], q_ready[NH]
+    static constexpr int NBARS = 4 + NKV + KSLOTS + VSLOTS + 7 * NH;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -118,15 +118,18 @@ __device__ __forceinline__ void produce_ring(const CUtensorMap* tm, uint8_t* rin
         if (!IS_K && n + 2 >= n_steps) mbar_arrive(bar);  // no K(n+2) exists
         mbar_arrive_expect_tx(bar, KB * KBOX);
         for (int kb = 0; kb < KB; ++kb)
-            tma_load_4d(ring + (slot * KB + kb) * KBOX, tm, bar, kb * 64, g, key_first - n * BN, b);
+            if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, (slot * KB + kb) * KBOX, KBOX, NS * KB * KBOX))
+                tma_load_4d(ring + (slot * KB + kb) * KBOX, tm, bar, kb * 64, g, key_first - n * BN, b);
         IRA_TRACE(p, trace_ev, n);
         last = n;
     }
     for (int n = (last >= NS ? last - NS + 1 : 0); n <= last; ++n)
-        mbar_wait_drain(bar_of(n), phase_of(n), p.timeout_ns);
+        mbar_wait_drain(bar_of(n), phase_of(n));
 }
 
-template <int D, int NH>
+// CLIP: the L2Clip of q is fused in (each softmax thread clips its row of the Q tile
+// in shared memory before the first product and stores the clipped row).
+template <int D, int NH, bool CLIP>
 __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const int num_qtiles) {
@@ -149,6 +152,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     uint64_t* p_full = s_full + 2 * NH;             // [NH][2]
     uint64_t* o_done = p_full + 2 * NH;             // [NH]
     uint64_t* o_full = o_done + NH;                 // [NH]
+    uint64_t* q_ready = o_full + NH;                // [NH]: Q of head s clipped (CLIP)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     CtaControl* ctl = reinterpret_cast<CtaControl*>(smem + L::MISC_OFF + 16);
     int* tinfo = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);
@@ -166,6 +170,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     const int i0 = qt * BM;
     const int i0g = p.q_off + i0;
     const int t64 = (p.S + 63) / 64;
+    // buffer extents for the bounds-checking build (elements; shared memory in bytes)
+    [[maybe_unused]] const uint32_t smem_base = smem_u32(smem);
+    [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -183,11 +190,14 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
             mbar_init(&p_full[2 * s + 1], 4);
             mbar_init(&o_done[s], 1);
             mbar_init(&o_full[s], 1);
+            mbar_init(&q_ready[s], 4);  // the head's softmax warps
         }
         ctl->abort = 0;
         const TileBounds* tb = p.tile_bounds + size_t(b) * t64 + 2 * qt;
-        int min_lo = tb[0].min_lo, max_hi = tb[0].max_hi, ne = tb[0].n_nonempty;
-        if (2 * qt + 1 < t64) {
+        const bool tb_ok = IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, size_t(b) * t64 + 2 * qt,
+                                         (2 * qt + 1 < t64) ? 2 : 1, (long long)p.B * t64);
+        int min_lo = tb_ok ? tb[0].min_lo : 0, max_hi = tb_ok ? tb[0].max_hi : -1, ne = tb_ok ? tb[0].n_nonempty : 0;
+        if (tb_ok && 2 * qt + 1 < t64) {
             min_lo = min(min_lo, tb[1].min_lo);
             max_hi = max(max_hi, tb[1].max_hi);
             ne += tb[1].n_nonempty;
@@ -233,7 +243,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                         tma_load_4d(q_smem(s, kb), &tm_q, q_full, kb * 64, h0 + s, i0, b);
                 produce_ring<KSLOTS, KB, true>(&tm_k, smem + L::K_OFF, k_first, kv_ready, k_empty, n_steps, g, b,
                                                key0(0), ctl, p, kErrFwdKFree, 1);
-                mbar_wait_drain(q_full, 0, p.timeout_ns);
+                mbar_wait_drain(q_full, 0);
             }
         } else if (warp == V_WARP) {
             // -------------------------------------------------------- V producer
@@ -282,7 +292,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     mma_commit(&o_done[s]);
                     IRA_TRACE(p, 5 + s, n);
                 };
-                bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
+                bool ok = mbar_wait(CLIP ? &q_ready[s] : q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
                 for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
                     ok = mbar_wait(&k_first[n], 0, ctl, p.err, kErrFwdK, p.timeout_ns);
                     if (!ok) break;
@@ -313,7 +323,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 if (ok) mma_commit(&o_full[s]);
                 // wait for every MMA of both issuers before TMEM is released
                 mma_commit(drain);
-                mbar_wait_drain(drain, 0, p.timeout_ns);
+                mbar_wait_drain(drain, 0);
             }
         }
     } else {
@@ -326,10 +336,18 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         const int h = h0 + s;
         const int i = i0 + r;
         const bool row_in = i < p.S;
-        const int2 rb = row_in ? p.row_bounds[size_t(b) * p.S + i] : make_int2(kEmptyLo, kEmptyHi);
+        const int2 rb = row_in && IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, size_t(b) * p.S + i, 1, (long long)p.B * p.S)
+                            ? p.row_bounds[size_t(b) * p.S + i]
+                            : make_int2(kEmptyLo, kEmptyHi);
         const bool empty = rb.x > rb.y;
         // no sink array: no sink term (a logit of -inf)
-        const float sigma = !row_in ? 0.f : p.sink ? p.sink[b * p.sink_sb + i * p.sink_ss + h * p.sink_sh] : -INFINITY;
+        const int64_t sink_at = b * p.sink_sb + i * p.sink_ss + h * p.sink_sh;
+        const float sigma = !row_in ? 0.f
+                            : !p.sink ? -INFINITY
+                            : IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, sink_at, 1,
+                                            (p.B - 1) * p.sink_sb + (p.S - 1) * p.sink_ss + (p.Hq - 1) * p.sink_sh + 1)
+                                ? p.sink[sink_at]
+                                : 0.f;
         float m2 = sigma * kLog2e;  // running maximum, log2 units
         float l = 1.f;              // running denominator; the sink contributes exp(0)
         bool seen = false;          // some earlier step held an unmasked key of this row
@@ -339,8 +357,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         const int m_r = (r + 1) & 7;   // misalignment of the row's window start
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
-        const uint16_t* prof_row =
-            (p.R > 0 && row_in && !empty) ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R) : nullptr;
+        const size_t prof_at = ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R);
+        const uint16_t* prof_row = (p.R > 0 && row_in && !empty) ? p.profiles + prof_at : nullptr;
+        [[maybe_unused]] const long long prof_n = (long long)p.B * p.Hq * p.S * p.R;
         auto delta_of = [&](int n) { return BN * (u_begin + n) - BN; };
         // the warp's smallest distance is delta + 32 wq - 63: no profile entry if >= R
         auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - (BN - 1) < p.R; };
@@ -355,7 +374,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     const int d0 = x0 + 8 * q;
                     const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
                     const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                    cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                    if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, dst + 16u * q - smem_base, 16, L::TOTAL) &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, inb ? prof_at + d0 : 0, inb ? 8 : 0, prof_n))
+                        cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
                 }
             }
             cp_async_commit();
@@ -372,6 +393,57 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 }
             }
         };
+
+        if constexpr (CLIP) {
+            // L2Clip of this row of q (head h): z = x * scale, y = z * min(1, thr / |z|) * tau,
+            // rounded to BF16, written over the Q tile in shared memory (for the products)
+            // and to q_clipped (for the backward). The tile is 128-byte swizzled: 16-byte
+            // chunk c of a row of a 64-column box sits at chunk c ^ (r mod 8) of that row.
+            const bool q_ok = warp_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
+            const float* const sc = p.clip_scale ? p.clip_scale + size_t(h) * D : nullptr;
+            auto chunk_at = [&](int c) {  // chunk c (8 columns) of the row
+                return q_smem(s, c >> 3) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+            };
+            auto chunk_z = [&](int c, float (&z)[8]) {
+                const uint4 u = *reinterpret_cast<const uint4*>(chunk_at(c));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    z[2 * e] = bf16lo_to_f32(wv[e]);
+                    z[2 * e + 1] = bf16hi_to_f32(wv[e]);
+                }
+                if (sc) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) z[e] *= sc[8 * c + e];
+                }
+            };
+            if (q_ok) {
+                float ss = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 8; ++c) {
+                    float z[8];
+                    chunk_z(c, z);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(z[e], z[e], ss);
+                }
+                const float nrm = sqrtf(ss);
+                float f = (nrm > p.clip_thr) ? p.clip_thr / nrm : 1.f;
+                if (p.clip_tau && row_in) f *= p.clip_tau[size_t(b) * p.S + i];
+                uint16_t* const grow = p.q_clipped + ((size_t(b) * p.S + i) * p.Hq + h) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 8; ++c) {
+                    float z[8];
+                    chunk_z(c, z);
+                    const uint4 y = make_uint4(pack_bf16x2(z[0] * f, z[1] * f), pack_bf16x2(z[2] * f, z[3] * f),
+                                               pack_bf16x2(z[4] * f, z[5] * f), pack_bf16x2(z[6] * f, z[7] * f));
+                    *reinterpret_cast<uint4*>(chunk_at(c)) = y;
+                    if (row_in) *reinterpret_cast<uint4*>(grow + 8 * c) = y;
+                }
+                fence_proxy_async_smem();  // the tensor core reads these bytes next
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_ready[s]);
+        }
 
         issue_band(0);
         issue_band(1);
@@ -423,8 +495,10 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                         if (s == 0 && lane == 0) IRA_TRACE(p, 24 + wq, n);  // per-warp band ready (head A)
                         const uint32_t* words =
                             reinterpret_cast<const uint32_t*>(band0 + buf * BAND_BYTES + row_off) + g_r;
+                        const bool w_ok = IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, smem_u32(words) - smem_base, 33 * 4,
+                                                        L::TOTAL);
 #pragma unroll
-                        for (int q = 0; q < 33; ++q) w[q] = words[q];
+                        for (int q = 0; q < 33; ++q) w[q] = w_ok ? words[q] : 0u;
                         if (s == 0 && lane == 0) IRA_TRACE(p, 36 + wq, __uint_as_float(w[0]) == 12345.f ? n + 1 : n);
                     }
                     // allowed columns [c_lo, c_lo + c_span] (none for an empty row)
@@ -572,16 +646,21 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                         v.y = empty ? 0.f : __uint_as_float(o[4 * q + 1]) * inv_l;
                         v.z = empty ? 0.f : __uint_as_float(o[4 * q + 2]) * inv_l;
                         v.w = empty ? 0.f : __uint_as_float(o[4 * q + 3]) * inv_l;
-                        *reinterpret_cast<float4*>(stage + lane * SP + 4 * q) = v;
+                        if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, smem_u32(stage + lane * SP + 4 * q) - smem_base,
+                                          16, L::TOTAL))
+                            *reinterpret_cast<float4*>(stage + lane * SP + 4 * q) = v;
                     }
                     __syncwarp();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int rr = 4 * k + sr;           // row of this warp
                         const int ir = i0 + 32 * wq + rr;    // its query row
-                        const float4 v = *reinterpret_cast<const float4*>(stage + rr * SP + sc);
-                        if (ir < p.S) {
-                            const int64_t at = b * p.row_sb + ir * p.row_ss + h * p.row_sh + 32 * c4 + sc;
+                        const bool st_ok = IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, smem_u32(stage + rr * SP + sc) - smem_base,
+                                                         16, L::TOTAL);
+                        const float4 v = st_ok ? *reinterpret_cast<const float4*>(stage + rr * SP + sc)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                        const int64_t at = b * p.row_sb + ir * p.row_ss + h * p.row_sh + 32 * c4 + sc;
+                        if (ir < p.S && IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, at, 4, n_rows * D)) {
                             if (p.out_bf16) {
                                 *reinterpret_cast<uint2*>(p.out_bf16 + at) =
                                     make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
@@ -592,12 +671,13 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     }
                     __syncwarp();
                 }
-            } else if (row_in) {
+            } else if (row_in && IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, orow_at, D, n_rows * D)) {
                 for (int e = 0; e < D; e += 4) store4(e, make_float4(0.f, 0.f, 0.f, 0.f));
             }
-            if (row_in) {
+            const int64_t lse_at = b * p.lse_sb + i * p.lse_ss + h * p.lse_sh;
+            if (row_in && IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, lse_at, 1, n_rows)) {
                 const float lse = (empty || n_steps == 0) ? sigma : (m2 + log2f(l)) * kLn2;
-                p.lse[b * p.lse_sb + i * p.lse_ss + h * p.lse_sh] = lse;
+                p.lse[lse_at] = lse;
             }
         }
     }
@@ -611,11 +691,11 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     }
 }
 
-template <int D, int NH>
+template <int D, int NH, bool CLIP>
 cudaError_t launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                         const AttnParams& p, cudaStream_t st) {
     using L = Layout<D, NH>;
-    auto kern = fwd_kernel<D, NH>;
+    auto kern = fwd_kernel<D, NH, CLIP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     const int num_qtiles = (p.S + BM - 1) / BM;
@@ -630,12 +710,20 @@ cudaError_t launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const 
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const AttnParams& p, cudaStream_t st) {
     const bool pair = (p.Hq / p.Hkv) % 2 == 0;
-    if (p.D == 128) {
-        return pair ? fwdk::launch_impl<128, 2>(tm_q, tm_k, tm_v, p, st)
-                    : fwdk::launch_impl<128, 1>(tm_q, tm_k, tm_v, p, st);
+    if (p.q_clipped) {
+        if (p.D == 128) {
+            return pair ? fwdk::launch_impl<128, 2, true>(tm_q, tm_k, tm_v, p, st)
+                        : fwdk::launch_impl<128, 1, true>(tm_q, tm_k, tm_v, p, st);
+        }
+        return pair ? fwdk::launch_impl<64, 2, true>(tm_q, tm_k, tm_v, p, st)
+                    : fwdk::launch_impl<64, 1, true>(tm_q, tm_k, tm_v, p, st);
     }
-    return pair ? fwdk::launch_impl<64, 2>(tm_q, tm_k, tm_v, p, st)
-                : fwdk::launch_impl<64, 1>(tm_q, tm_k, tm_v, p, st);
+    if (p.D == 128) {
+        return pair ? fwdk::launch_impl<128, 2, false>(tm_q, tm_k, tm_v, p, st)
+                    : fwdk::launch_impl<128, 1, false>(tm_q, tm_k, tm_v, p, st);
+    }
+    return pair ? fwdk::launch_impl<64, 2, false>(tm_q, tm_k, tm_v, p, st)
+                : fwdk::launch_impl<64, 1, false>(tm_q, tm_k, tm_v, p, st);
 }
 
 }  // namespace ira

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "inkling_flex_attn.h"
+#include "inkling_l2clip.h"
 #include "inkling_rel_attn.h"
 #include "launch.h"
 
@@ -100,6 +101,10 @@ struct NvtxRange {
     NvtxRange(const NvtxRange&) = delete;
     NvtxRange& operator=(const NvtxRange&) = delete;
 };
+
+// Limit of the attention kernels' pipeline waits for later calls
+// (inkling_rel_attn_set_wait_timeout_ns); 0 = the default.
+uint64_t g_wait_timeout_ns = 0;
 
 // Optional per-launch timing events (inkling_rel_attn_set_timing_events).
 cudaEvent_t const* g_events = nullptr;
@@ -233,7 +238,7 @@ AttnParams base_params(const inkling_rel_attn_dims* d, const Ws& w, const uint16
     p.q_off = int(d->query_offset);
     p.scale = 1.0f / sqrtf(float(d->head_dim));
     p.scale_log2 = p.scale * kLog2e;
-    p.timeout_ns = kDefaultTimeoutNs;
+    p.timeout_ns = g_wait_timeout_ns ? g_wait_timeout_ns : kDefaultTimeoutNs;
     p.profiles = profiles;
     p.safe_src = w.row_bounds();
     p.sink = sink;
@@ -275,25 +280,67 @@ inkling_status run_bounds(const inkling_rel_attn_dims* d, const Ws& w, const uin
     return cuda_status(e);
 }
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device (with that device current) and cached.
-constexpr int kMaxDevices = 64;
+// Device address of g_noalloc_scratch in the calling thread's current CUDA
+// context, looked up once per context (with that context current) and cached.
+// The cache is keyed by the context's process-unique id (cuCtxGetId), so a
+// context created after cudaDeviceReset, or a non-primary context made current
+// by the caller, gets its own lookup instead of a stale address.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+struct NoAllocSlot {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+constexpr int kNoAllocSlots = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
+NoAllocSlot g_noalloc_slots[kNoAllocSlots] = {};
+int g_noalloc_used = 0;
+
+inkling_status current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return INKLING_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return INKLING_ERR_CUDA;
+    if (!ctx) {
+        // no context on this thread yet: a runtime call that needs one makes the
+        // current device's primary context current (and allocates nothing)
+        void* p = nullptr;
+        if (note(cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return INKLING_ERR_CUDA;
+        if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return INKLING_ERR_CUDA;
+    }
+    return get_id(ctx, id) == CUDA_SUCCESS ? INKLING_OK : INKLING_ERR_CUDA;
+}
 
 inkling_status noalloc_scratch(void** out) {
-    int dev = -1;
-    cudaError_t e = note(cudaGetDevice(&dev));
-    if (e != cudaSuccess) return INKLING_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return INKLING_ERR_UNSUPPORTED;
+    unsigned long long id = 0;
+    inkling_status s = current_context_id(&id);
+    if (s != INKLING_OK) return s;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        e = note(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-        if (e != cudaSuccess || !p) return INKLING_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    for (int k = 0; k < g_noalloc_used; ++k)
+        if (g_noalloc_slots[k].ctx_id == id) {
+            *out = g_noalloc_slots[k].ptr;
+            return INKLING_OK;
+        }
+    void* p = nullptr;
+    cudaError_t e = note(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (e != cudaSuccess || !p) return INKLING_ERR_CUDA;
+    // a full table is refilled from the start (its entries only save lookups)
+    if (g_noalloc_used == kNoAllocSlots) g_noalloc_used = 0;
+    g_noalloc_slots[g_noalloc_used++] = NoAllocSlot{id, p};
+    *out = p;
     return INKLING_OK;
 }
 
@@ -451,6 +498,171 @@ cudaError_t flex_masks(const inkling_flex_attn_dims* f, const int64_t* tokens, c
     return note(e);
 }
 
+// L2Clip of q fused into the attention (the *_qclip entry points).
+struct QClipArgs {
+    float thr;
+    const float* scale;         // [Hq, D] or null
+    const float* tau;           // [B, S] or null
+    uint16_t* q_clipped;        // forward: the clipped q (written)
+    const uint16_t* q_raw;      // backward: the unclipped q
+    float* dscale;              // backward: gradient of scale (or null)
+    float* dtau;                // backward: gradient of tau (or null)
+};
+
+// Backward workspace of the fused path: the ordinary one, then the dQ kernel's parts of
+// dscale [B * ceil(S / 128)][Hq][D] and of dtau [B, S, Hq].
+struct QClipLayout {
+    size_t dscale_part, dtau_part, total;
+    int64_t nchunks;
+};
+QClipLayout qclip_layout(const inkling_rel_attn_dims* d) {
+    QClipLayout q{};
+    const size_t base = workspace_layout(d->batch, d->seq_q, d->heads_q, d->head_dim, true).total;
+    q.nchunks = d->batch * ((d->seq_q + 127) / 128);
+    q.dscale_part = align_up(base, 256);
+    q.dtau_part = align_up(q.dscale_part + size_t(q.nchunks) * d->heads_q * d->head_dim * 4, 256);
+    q.total = align_up(q.dtau_part + size_t(d->batch) * d->seq_q * d->heads_q * 4, 256);
+    return q;
+}
+
+// The forward of either ABI; `qc` (optional) fuses the L2Clip of q in: q is then the
+// unclipped q, and the clipped q is stored to qc->q_clipped.
+inkling_status fwd_impl(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* profiles, const float* sink, const uint8_t* valid, const uint8_t* key_valid,
+                        const int32_t* positions, const int32_t* key_positions, float* out, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream, const QClipArgs* qc) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
+    if (nq > 0 && (!q || !sink || !valid || !out || !lse)) return INKLING_ERR_INVALID_ARG;
+    if (nq > 0 && dims->rel_extent > 0 && !profiles) return INKLING_ERR_INVALID_ARG;
+    if (nk > 0 && (!k || !v)) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out))
+        return INKLING_ERR_INVALID_ARG;
+    int kpq = 0;
+    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
+    if (s != INKLING_OK) return s;
+    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
+    Ws w;
+    s = get_ws(dims, false, workspace, workspace_bytes, &w);
+    if (s != INKLING_OK) return s;
+    if (nq == 0) return INKLING_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // K/V maps need at least one row; with no keys every row is empty and the
+    // kernel never reads them, so point them at q.
+    const bool no_keys = dims->seq_k == 0;
+    CUtensorMap tq, tk, tv;
+    if (!encode_bhtd(&tq, q, dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, 128) ||
+        !encode_bhtd(&tk, no_keys ? q : k, dims->batch, no_keys ? 1 : dims->seq_k,
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64) ||
+        !encode_bhtd(&tv, no_keys ? q : v, dims->batch, no_keys ? 1 : dims->seq_k,
+                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64))
+        return INKLING_ERR_CUDA;
+
+    LaunchTimer tm(st);
+    s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
+    if (s != INKLING_OK) return s;
+    AttnParams p = base_params(dims, w, profiles, sink);
+    p.out = out;
+    p.lse = lse;
+    if (qc) {
+        p.clip_thr = qc->thr;
+        p.clip_scale = qc->scale;
+        p.clip_tau = qc->tau;
+        p.q_clipped = qc->q_clipped;
+    }
+    return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+}
+
+// The backward of either ABI; `qc` (optional) fuses the L2Clip backward of q in: q is
+// then the clipped q the forward stored, dq receives the gradient of the unclipped q
+// (qc->q_raw), and qc->dscale / qc->dtau (when set) the clip's parameter gradients.
+inkling_status bwd_impl(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* profiles, const float* sink, const uint8_t* valid, const uint8_t* key_valid,
+                        const int32_t* positions, const int32_t* key_positions, const float* out, const float* lse,
+                        const float* dout, const float* dlse, float* dq, float* dk, float* dv, float* dprofiles,
+                        float* dsink, void* workspace, size_t workspace_bytes, void* stream, const QClipArgs* qc) {
+    inkling_status s = check_dims(dims);
+    if (s != INKLING_OK) return s;
+    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
+    if (nq > 0 && (!q || !sink || !valid || !out || !lse || !dout || !dq || !dsink)) return INKLING_ERR_INVALID_ARG;
+    if (nq > 0 && dims->rel_extent > 0 && (!profiles || !dprofiles)) return INKLING_ERR_INVALID_ARG;
+    if (nk > 0 && (!k || !v || !dk || !dv)) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dprofiles))
+        return INKLING_ERR_INVALID_ARG;
+    int kpq = 0;
+    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
+    if (s != INKLING_OK) return s;
+    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
+    Ws w;
+    s = get_ws(dims, true, workspace, workspace_bytes, &w);
+    if (s != INKLING_OK) return s;
+    const QClipLayout ql = qclip_layout(dims);
+    if (qc && workspace_bytes < ql.total) return INKLING_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (nq == 0) {
+        // no queries: every key gradient is zero, and so is the clip's scale gradient
+        cudaError_t e = cudaSuccess;
+        if (nk > 0) {
+            const size_t bytes = size_t(nk) * dims->heads_kv * dims->head_dim * 4;
+            e = cudaMemsetAsync(dk, 0, bytes, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, st);
+        }
+        if (e == cudaSuccess && qc && qc->dscale)
+            e = cudaMemsetAsync(qc->dscale, 0, size_t(dims->heads_q) * dims->head_dim * 4, st);
+        return cuda_status(e);
+    }
+    const bool no_keys = dims->seq_k == 0;
+    auto* dout_bf16 = reinterpret_cast<__nv_bfloat16*>(w.base + w.L.dout_bf16);
+    auto* lse2t = reinterpret_cast<float*>(w.base + w.L.lse2t);
+    auto* dvt = reinterpret_cast<float*>(w.base + w.L.dvt);
+    CUtensorMap tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64;
+    const int64_t B = dims->batch, S = dims->seq_q, Hq = dims->heads_q, D = dims->head_dim;
+    const int64_t Skv_m = no_keys ? 1 : dims->seq_k, Hkv_m = no_keys ? Hq : dims->heads_kv;
+    const void* kb = no_keys ? static_cast<const void*>(q) : k;
+    const void* vb = no_keys ? static_cast<const void*>(q) : v;
+    if (!encode_bhtd(&tq64, q, B, S, Hq, D, 64) || !encode_bhtd(&tq128, q, B, S, Hq, D, 128) ||
+        !encode_bhtd(&tdo64, dout_bf16, B, S, Hq, D, 64) || !encode_bhtd(&tdo128, dout_bf16, B, S, Hq, D, 128) ||
+        !encode_bhtd(&tk128, kb, B, Skv_m, Hkv_m, D, 128) || !encode_bhtd(&tv128, vb, B, Skv_m, Hkv_m, D, 128) ||
+        !encode_bhtd(&tk64, kb, B, Skv_m, Hkv_m, D, 64) || !encode_bhtd(&tv64, vb, B, Skv_m, Hkv_m, D, 64))
+        return INKLING_ERR_CUDA;
+    CUtensorMap tband;
+    std::memset(&tband, 0, sizeof(tband));
+    if (dims->rel_extent > 0 && !encode_band(&tband, profiles, B * Hq * S, dims->rel_extent)) return INKLING_ERR_CUDA;
+
+    AttnParams p = base_params(dims, w, profiles, sink);
+    p.lse2t = lse2t;
+    p.dvt = dvt;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dprofiles = dprofiles;
+    float* dscale_part = nullptr;
+    float* dtau_part = nullptr;
+    if (qc) {
+        dscale_part = reinterpret_cast<float*>(w.base + ql.dscale_part);
+        dtau_part = reinterpret_cast<float*>(w.base + ql.dtau_part);
+        p.clip_thr = qc->thr;
+        p.clip_scale = qc->scale;
+        p.clip_tau = qc->tau;
+        p.q_raw = qc->q_raw;
+        p.dscale_part = dscale_part;
+        p.dtau_part = dtau_part;
+    }
+    BwdMaps mp{tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64, tband};
+    s = bwd_launches(dims, w, p, mp, valid, key_valid, positions, nk > 0, st, nullptr,
+                     [&](cudaStream_t s0) {
+                         return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq),
+                                                dsink, dout_bf16, lse2t, dvt, s0);
+                     });
+    if (s != INKLING_OK || !qc || (!qc->dscale && !qc->dtau)) return s;
+    // the clip's parameter gradients: sums of the dQ kernel's parts, in a fixed order
+    return cuda_status(launch_l2clip_reduce(dtau_part, B * S, int(Hq), qc->dtau, dscale_part, ql.nchunks, Hq * D,
+                                            qc->dscale, st));
+}
+
 }  // namespace
 
 namespace ira {
@@ -512,42 +724,8 @@ inkling_status inkling_rel_attn_fwd(const inkling_rel_attn_dims* dims, const uin
                                     const int32_t* key_positions, float* out, float* lse, void* workspace,
                                     size_t workspace_bytes, void* stream) {
     NvtxRange nvtx_range("inkling_rel_attn_fwd");
-    inkling_status s = check_dims(dims);
-    if (s != INKLING_OK) return s;
-    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
-    if (nq > 0 && (!q || !sink || !valid || !out || !lse)) return INKLING_ERR_INVALID_ARG;
-    if (nq > 0 && dims->rel_extent > 0 && !profiles) return INKLING_ERR_INVALID_ARG;
-    if (nk > 0 && (!k || !v)) return INKLING_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out))
-        return INKLING_ERR_INVALID_ARG;
-    int kpq = 0;
-    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
-    if (s != INKLING_OK) return s;
-    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
-    Ws w;
-    s = get_ws(dims, false, workspace, workspace_bytes, &w);
-    if (s != INKLING_OK) return s;
-    if (nq == 0) return INKLING_OK;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-    // K/V maps need at least one row; with no keys every row is empty and the
-    // kernel never reads them, so point them at q.
-    const bool no_keys = dims->seq_k == 0;
-    CUtensorMap tq, tk, tv;
-    if (!encode_bhtd(&tq, q, dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, 128) ||
-        !encode_bhtd(&tk, no_keys ? q : k, dims->batch, no_keys ? 1 : dims->seq_k,
-                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64) ||
-        !encode_bhtd(&tv, no_keys ? q : v, dims->batch, no_keys ? 1 : dims->seq_k,
-                     no_keys ? dims->heads_q : dims->heads_kv, dims->head_dim, 64))
-        return INKLING_ERR_CUDA;
-
-    LaunchTimer tm(st);
-    s = run_bounds(dims, w, valid, key_valid, positions, st, tm);
-    if (s != INKLING_OK) return s;
-    AttnParams p = base_params(dims, w, profiles, sink);
-    p.out = out;
-    p.lse = lse;
-    return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+    return fwd_impl(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, workspace,
+                    workspace_bytes, stream, nullptr);
 }
 
 inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
@@ -558,64 +736,58 @@ inkling_status inkling_rel_attn_bwd(const inkling_rel_attn_dims* dims, const uin
                                     float* dprofiles, float* dsink, void* workspace, size_t workspace_bytes,
                                     void* stream) {
     NvtxRange nvtx_range("inkling_rel_attn_bwd");
-    inkling_status s = check_dims(dims);
-    if (s != INKLING_OK) return s;
-    const int64_t nq = dims->batch * dims->seq_q, nk = dims->batch * dims->seq_k;
-    if (nq > 0 && (!q || !sink || !valid || !out || !lse || !dout || !dq || !dsink)) return INKLING_ERR_INVALID_ARG;
-    if (nq > 0 && dims->rel_extent > 0 && (!profiles || !dprofiles)) return INKLING_ERR_INVALID_ARG;
-    if (nk > 0 && (!k || !v || !dk || !dv)) return INKLING_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(profiles) || !aligned16(out) ||
-        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dprofiles))
-        return INKLING_ERR_INVALID_ARG;
-    int kpq = 0;
-    s = resolve_key_side(dims, valid, key_valid, positions, key_positions, &kpq);
-    if (s != INKLING_OK) return s;
-    if (nk > 0 && !key_valid) return INKLING_ERR_INVALID_ARG;
-    Ws w;
-    s = get_ws(dims, true, workspace, workspace_bytes, &w);
-    if (s != INKLING_OK) return s;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (nq == 0) {
-        // no queries: every key gradient is zero
-        cudaError_t e = cudaSuccess;
-        if (nk > 0) {
-            const size_t bytes = size_t(nk) * dims->heads_kv * dims->head_dim * 4;
-            e = cudaMemsetAsync(dk, 0, bytes, st);
-            if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, st);
-        }
-        return cuda_status(e);
-    }
-    const bool no_keys = dims->seq_k == 0;
-    auto* dout_bf16 = reinterpret_cast<__nv_bfloat16*>(w.base + w.L.dout_bf16);
-    auto* lse2t = reinterpret_cast<float*>(w.base + w.L.lse2t);
-    auto* dvt = reinterpret_cast<float*>(w.base + w.L.dvt);
-    CUtensorMap tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64;
-    const int64_t B = dims->batch, S = dims->seq_q, Hq = dims->heads_q, D = dims->head_dim;
-    const int64_t Skv_m = no_keys ? 1 : dims->seq_k, Hkv_m = no_keys ? Hq : dims->heads_kv;
-    const void* kb = no_keys ? static_cast<const void*>(q) : k;
-    const void* vb = no_keys ? static_cast<const void*>(q) : v;
-    if (!encode_bhtd(&tq64, q, B, S, Hq, D, 64) || !encode_bhtd(&tq128, q, B, S, Hq, D, 128) ||
-        !encode_bhtd(&tdo64, dout_bf16, B, S, Hq, D, 64) || !encode_bhtd(&tdo128, dout_bf16, B, S, Hq, D, 128) ||
-        !encode_bhtd(&tk128, kb, B, Skv_m, Hkv_m, D, 128) || !encode_bhtd(&tv128, vb, B, Skv_m, Hkv_m, D, 128) ||
-        !encode_bhtd(&tk64, kb, B, Skv_m, Hkv_m, D, 64) || !encode_bhtd(&tv64, vb, B, Skv_m, Hkv_m, D, 64))
-        return INKLING_ERR_CUDA;
-    CUtensorMap tband;
-    std::memset(&tband, 0, sizeof(tband));
-    if (dims->rel_extent > 0 && !encode_band(&tband, profiles, B * Hq * S, dims->rel_extent)) return INKLING_ERR_CUDA;
+    return bwd_impl(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout, dlse,
+                    dq, dk, dv, dprofiles, dsink, workspace, workspace_bytes, stream, nullptr);
+}
 
-    AttnParams p = base_params(dims, w, profiles, sink);
-    p.lse2t = lse2t;
-    p.dvt = dvt;
-    p.dq = dq;
-    p.dk = dk;
-    p.dv = dv;
-    p.dprofiles = dprofiles;
-    BwdMaps mp{tq64, tq128, tdo64, tdo128, tk128, tv128, tk64, tv64, tband};
-    return bwd_launches(dims, w, p, mp, valid, key_valid, positions, nk > 0, st, nullptr,
-                        [&](cudaStream_t s0) {
-                            return launch_bwd_prep(int(D), out, lse, sink, dout, dlse, int(B), int(S), int(Hq),
-                                                   dsink, dout_bf16, lse2t, dvt, s0);
-                        });
+size_t inkling_rel_attn_qclip_workspace_size(const inkling_rel_attn_dims* dims, int backward) {
+    if (check_dims(dims) != INKLING_OK) return 0;
+    return backward ? qclip_layout(dims).total
+                    : workspace_layout(dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, false).total;
+}
+
+inkling_status inkling_rel_attn_fwd_qclip(const inkling_rel_attn_dims* dims, double threshold, const float* clip_scale,
+                                          const float* tau, const uint16_t* x, const uint16_t* k, const uint16_t* v,
+                                          const uint16_t* profiles, const float* sink, const uint8_t* valid,
+                                          const uint8_t* key_valid, const int32_t* positions,
+                                          const int32_t* key_positions, uint16_t* q_clipped, float* out, float* lse,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("inkling_rel_attn_fwd_qclip");
+    if (!(threshold >= 0.0) || !std::isfinite(threshold)) return INKLING_ERR_INVALID_ARG;
+    if (dims && dims->batch * dims->seq_q > 0 && !q_clipped) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(q_clipped) || !aligned16(x)) return INKLING_ERR_INVALID_ARG;
+    QClipArgs qc{};
+    qc.thr = float(threshold);
+    qc.scale = clip_scale;
+    qc.tau = tau;
+    qc.q_clipped = q_clipped;
+    return fwd_impl(dims, x, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, workspace,
+                    workspace_bytes, stream, &qc);
+}
+
+inkling_status inkling_rel_attn_bwd_qclip(const inkling_rel_attn_dims* dims, double threshold, const float* clip_scale,
+                                          const float* tau, const uint16_t* x, const uint16_t* q_clipped,
+                                          const uint16_t* k, const uint16_t* v, const uint16_t* profiles,
+                                          const float* sink, const uint8_t* valid, const uint8_t* key_valid,
+                                          const int32_t* positions, const int32_t* key_positions, const float* out,
+                                          const float* lse, const float* dout, const float* dlse, float* dx, float* dk,
+                                          float* dv, float* dprofiles, float* dsink, float* dclip_scale, float* dtau,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx_range("inkling_rel_attn_bwd_qclip");
+    if (!(threshold >= 0.0) || !std::isfinite(threshold)) return INKLING_ERR_INVALID_ARG;
+    if (dims && dims->batch * dims->seq_q > 0 && !x) return INKLING_ERR_INVALID_ARG;
+    if ((dclip_scale != nullptr) != (clip_scale != nullptr) || (dtau != nullptr) != (tau != nullptr))
+        return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(x)) return INKLING_ERR_INVALID_ARG;
+    QClipArgs qc{};
+    qc.thr = float(threshold);
+    qc.scale = clip_scale;
+    qc.tau = tau;
+    qc.q_raw = x;
+    qc.dscale = dclip_scale;
+    qc.dtau = dtau;
+    return bwd_impl(dims, q_clipped, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse, dout,
+                    dlse, dx, dk, dv, dprofiles, dsink, workspace, workspace_bytes, stream, &qc);
 }
 
 inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, const uint16_t* q, const uint16_t* k,
@@ -623,6 +795,7 @@ inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, c
                                             const uint8_t* valid, const uint8_t* key_valid,
                                             const int32_t* positions, const int32_t* key_positions, float* out,
                                             float* lse, void* stream) {
+    NvtxRange nvtx_range("inkling_rel_attn_fwd_noalloc");
     inkling_status s = check_dims(dims);
     if (s != INKLING_OK) return s;
     if (workspace_layout(dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, false).total >
@@ -635,6 +808,14 @@ inkling_status inkling_rel_attn_fwd_noalloc(const inkling_rel_attn_dims* dims, c
     // device error word itself and rewrites every other scratch byte it reads)
     return inkling_rel_attn_fwd(dims, q, k, v, profiles, sink, valid, key_valid, positions, key_positions, out, lse,
                                 scratch, kNoAllocScratchBytes, stream);
+}
+
+inkling_status inkling_rel_attn_fwd_noalloc_last_device_error(void* stream) {
+    void* scratch = nullptr;
+    inkling_status s = noalloc_scratch(&scratch);
+    if (s != INKLING_OK) return s;
+    // the device error word sits at the start of the array, as in any workspace
+    return inkling_rel_attn_last_device_error(scratch, stream);
 }
 
 size_t inkling_flex_attn_workspace_size(const inkling_flex_attn_dims* dims, int backward) {
@@ -730,6 +911,15 @@ inkling_status inkling_flex_attn_bwd(const inkling_flex_attn_dims* dims, const u
         });
 }
 
+inkling_status inkling_rel_attn_merge(int64_t rows, int64_t head_dim, float* out, float* lse, const float* out_part,
+                                      const float* lse_part, void* stream) {
+    NvtxRange nvtx_range("inkling_rel_attn_merge");
+    if (rows < 0 || (head_dim != 64 && head_dim != 128)) return INKLING_ERR_INVALID_ARG;
+    if (rows > 0 && (!out || !lse || !out_part || !lse_part)) return INKLING_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(out_part)) return INKLING_ERR_INVALID_ARG;
+    return cuda_status(launch_merge(out, lse, out_part, lse_part, rows, int(head_dim), static_cast<cudaStream_t>(stream)));
+}
+
 inkling_status inkling_rel_attn_last_device_error(void* workspace, void* stream) {
     if (!workspace) return INKLING_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -759,6 +949,11 @@ inkling_status inkling_rel_attn_selftest_wait_timeout(uint32_t timeout_us, void*
 inkling_status inkling_rel_attn_selftest_exp2(const float* t, float* out, int64_t n, void* stream) {
     if (n < 0 || (n > 0 && (!t || !out)) || n > (int64_t(1) << 40)) return INKLING_ERR_INVALID_ARG;
     return cuda_status(note(launch_selftest_exp2(t, out, n, static_cast<cudaStream_t>(stream))));
+}
+
+inkling_status inkling_rel_attn_set_wait_timeout_ns(uint64_t timeout_ns) {
+    g_wait_timeout_ns = timeout_ns;
+    return INKLING_OK;
 }
 
 inkling_status inkling_rel_attn_set_timing_events(void* const* events, int n_pairs) {

@@ -282,6 +282,20 @@ inkling_status status_of(cudaError_t e) { return ira::note_cuda_error(e) == cuda
 
 }  // namespace
 
+namespace ira {
+// dtau[t] = sum over h of dtau_part[t, h] (t < T) and dscale[j] = sum over chunks of
+// dscale_part[chunk, j] (j < HD), in a fixed order; either output may be null. Used by the
+// L2Clip of q fused into the attention backward as well.
+cudaError_t launch_l2clip_reduce(const float* dtau_part, int64_t T, int H, float* dtau, const float* dscale_part,
+                                 int64_t nchunks, int64_t HD, float* dscale, cudaStream_t st) {
+    const int64_t n = T + HD;
+    if (n == 0) return cudaSuccess;
+    l2clip_reduce_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(dtau_part, T, H, dtau, dscale_part, nchunks, HD,
+                                                                   dscale);
+    return cudaGetLastError();
+}
+}  // namespace ira
+
 extern "C" {
 
 size_t inkling_l2clip_workspace_size(const inkling_l2clip_dims* dims) {

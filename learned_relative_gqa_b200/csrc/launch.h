@@ -21,6 +21,10 @@ cudaError_t launch_bwd_prep(int D, const float* out, const float* lse, const flo
 cudaError_t launch_dprof_zero(const int2* row_bounds, int B, int S, int Hq, int R, int q_off, float* dprof,
                               cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, int* err, cudaStream_t st);
+// Context parallelism: merges a partial result (out_part, lse_part) over a disjoint key
+// set into (out, lse), rows = B * S * Hq of D floats.
+cudaError_t launch_merge(float* out, float* lse, const float* out_part, const float* lse_part, int64_t rows, int D,
+                         cudaStream_t st);
 
 // Generic FlexAttention variant: block positions from EOS tokens / fixed blocks, the
 // backward preprocessing of BF16 [B, H, S, D] out / dout rows, and the per-head sum of
@@ -33,6 +37,10 @@ cudaError_t launch_flex_bwd_prep(int D, const uint16_t* out, const uint16_t* dou
 cudaError_t launch_flex_dsink_reduce(const float* dsink_rows, int B, int S, int Hq, float* dsink_weights,
                                      cudaStream_t st);
 cudaError_t launch_selftest_exp2(const float* t, float* out, int64_t n, cudaStream_t st);
+// L2Clip backward reduction (l2clip.cu): dtau[t] = sum_h dtau_part[t, h], dscale[j] = sum
+// over chunks of dscale_part[chunk, j]; fixed order, null outputs skipped.
+cudaError_t launch_l2clip_reduce(const float* dtau_part, int64_t T, int H, float* dtau, const float* dscale_part,
+                                 int64_t nchunks, int64_t HD, float* dscale, cudaStream_t st);
 
 // Forward attention. tm_q: {D, Hq, S, B} box {64,1,128,1}; tm_k / tm_v: {D, Hkv, Skv, B} box {64,1,64,1}.
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,

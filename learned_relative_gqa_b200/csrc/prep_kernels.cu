@@ -15,6 +15,8 @@
 // (positions restart at every document, per the Inkling2FlexAttention.forward
 // page), so the interval is exactly the causal, same-document, in-window,
 // valid keys of the definition.
+#include <algorithm>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -37,6 +39,44 @@ __device__ __forceinline__ int warp_max(int v) {
 __device__ __forceinline__ int warp_sum(int v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// Merge of two results for the same query rows over disjoint key sets (context
+// parallelism: the local keys first, the keys of the ranks before later), each
+// normalised over its own keys with its own log-sum-exp:
+//   lse = log(exp(lse_a) + exp(lse_b)),
+//   out = out_a exp(lse_a - lse) + out_b exp(lse_b - lse),
+// written over (out_a, lse_a). One warp per row, float4 accesses. A row whose
+// parts are both empty (both lse -inf) keeps out = 0 and lse = -inf.
+__global__ void merge_kernel(float* __restrict__ out_a, float* __restrict__ lse_a, const float* __restrict__ out_b,
+                             const float* __restrict__ lse_b, int64_t rows, int D) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+        const float la = lse_a[r], lb = lse_b[r];
+        const float m = fmaxf(la, lb);
+        float wa = 0.f, wb = 0.f, l = m;
+        if (m > -INFINITY) {
+            const float ea = expf(la - m), eb = expf(lb - m);
+            const float sum = ea + eb;
+            wa = ea / sum;
+            wb = eb / sum;
+            l = m + logf(sum);
+        }
+        float4* oa = reinterpret_cast<float4*>(out_a + r * D);
+        const float4* ob = reinterpret_cast<const float4*>(out_b + r * D);
+        for (int c = lane; c < D / 4; c += 32) {
+            float4 x = oa[c];
+            const float4 y = ob[c];
+            x.x = fmaf(x.x, wa, y.x * wb);
+            x.y = fmaf(x.y, wa, y.y * wb);
+            x.z = fmaf(x.z, wa, y.z * wb);
+            x.w = fmaf(x.w, wa, y.w * wb);
+            oa[c] = x;
+        }
+        __syncwarp();
+        if (lane == 0) lse_a[r] = l;
+    }
 }
 
 }  // namespace
@@ -455,6 +495,14 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ t, float* __restr
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
+cudaError_t launch_merge(float* out, float* lse, const float* out_part, const float* lse_part, int64_t rows, int D,
+                         cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((rows + 7) / 8, 148 * 16);
+    merge_kernel<<<unsigned(blocks), 256, 0, st>>>(out, lse, out_part, lse_part, rows, D);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_kspan(const uint8_t* key_valid, int B, int Skv, int2* kspan, cudaStream_t st) {
     if (B == 0) return cudaSuccess;
     kspan_kernel<<<B, 512, 0, st>>>(key_valid, Skv, kspan);

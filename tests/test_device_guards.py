@@ -37,6 +37,33 @@ def test_normal_calls_leave_no_device_error():
     assert binding.inkling_rel_attn_last_device_error(ws) == binding.INKLING_OK
 
 
+def test_forward_abort_path_reports_a_timeout_and_the_context_survives():
+    """With the pipeline waits limited to 1 ns, a CTA's first wait that does not
+    succeed at once (its MMA issuer's wait for the Q tile) runs out: the CTA records
+    the site, stops every role, drains its copies and products with the default limit
+    and exits. The call reports the timeout; the same call with the default limit then
+    completes and matches the oracle, so the context is intact."""
+    x = W.make_inputs(U.custom("abort", 1, 256, 4, 2, 128, 0, 64, docs=(40, 200)), "cuda")
+    dims = binding.make_dims(x["q"], x["k"], x["profiles"], 0)
+    ws = binding.alloc_workspace(dims, False, "cuda")
+    args = (x["q"], x["k"], x["v"], x["profiles"], x["sink"], x["valid"], x["key_valid"], x["positions"],
+            x["key_positions"])
+    binding.inkling_rel_attn_set_wait_timeout_ns(1)
+    try:
+        binding.forward(*args, workspace=ws)
+        torch.cuda.synchronize()
+        st = binding.inkling_rel_attn_last_device_error(ws)
+    finally:
+        binding.inkling_rel_attn_set_wait_timeout_ns(0)
+    assert st == binding.INKLING_ERR_TIMEOUT
+    out, lse = binding.forward(*args, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.inkling_rel_attn_last_device_error(ws) == binding.INKLING_OK
+    o_ref, l_ref, _ = U.oracle_forward(U.to_host(x))
+    U.assert_out_close(out.cpu().numpy(), o_ref)
+    U.assert_lse_close(lse.cpu().numpy(), l_ref)
+
+
 def _validate(x):
     dims = binding.make_dims(x["q"], x["k"], x["profiles"], x["window"], x["query_offset"])
     ws = binding.alloc_workspace(dims, False, "cuda")

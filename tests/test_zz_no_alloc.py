@@ -5,7 +5,9 @@ buffers from their host framework, or may not call cudaMalloc because it can
 synchronise the device). inkling_rel_attn_fwd_noalloc serves them with scratch
 held in a static device array inside the library. This file runs last (pytest
 collects it after the others) and checks, through the C ABI, that two calls in
-a row agree with the ordinary workspace-taking forward.
+a row agree with the ordinary workspace-taking forward, that a call leaves the
+device's free memory and PyTorch's allocation count unchanged, and that the
+entry point's own device error word reads back clean.
 """
 import pytest
 import torch
@@ -28,14 +30,22 @@ def test_noalloc_forward_matches_workspace_forward_twice():
     x = W.make_inputs(w, "cuda")
     ref_out, ref_lse = U.gpu_forward(x)
     dims = binding.make_dims(x["q"], x["k"], x["profiles"], x["window"], x["query_offset"])
-    for _ in range(2):
+    for call in range(2):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
+        torch.cuda.synchronize()
+        # the first call loads the library's module and looks its scratch up; from the
+        # second on, a call must not change the device's free memory at all
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         st = binding.inkling_rel_attn_fwd_noalloc(dims, x["q"], x["k"], x["v"], x["profiles"], x["sink"],
                                                   x["valid"], x["key_valid"], x["positions"], x["key_positions"],
                                                   out, lse)
         assert st == binding.INKLING_OK
         torch.cuda.synchronize()
+        if call > 0:
+            assert torch.cuda.mem_get_info()[0] == free0, "the no-allocation forward changed free device memory"
+            assert torch.cuda.memory_allocated() == alloc0
+        assert binding.inkling_rel_attn_fwd_noalloc_last_device_error() == binding.INKLING_OK
         U.assert_out_close(out.cpu().numpy(), ref_out.cpu().double().numpy(), "noalloc out")
         U.assert_lse_close(lse.cpu().numpy(), ref_lse.cpu().double().numpy(), "noalloc lse")
 
