@@ -489,6 +489,8 @@ def main():
     ap.add_argument("--flex-steps", type=int, default=3,
                     help="forward + backward steps of the generic FlexAttention variant (0 = skip)")
     ap.add_argument("--l2clip-steps", type=int, default=5, help="L2Clip forward + backward steps (0 = skip)")
+    ap.add_argument("--qclip-steps", type=int, default=-1,
+                    help="steps of the workload with the L2Clip of q fused in, and with it separate (-1: as l2clip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-csv-dir", default="/tmp",
                     help="directory for the CSV of the SM clock samples taken during the timed regions")
@@ -635,6 +637,11 @@ def main():
     l2c = None
     if args.l2clip_steps > 0 and rank == 0:
         l2c = l2clip_run(args.l2clip_steps, device, peaks)
+    qclip_steps = args.l2clip_steps if args.qclip_steps < 0 else args.qclip_steps
+    if qclip_steps > 0 and rank == 0 and backward:
+        torch.cuda.empty_cache()
+        fused = qclip_run(qclip_steps, device, peaks, w)
+        l2c = dict(l2c or {}, fused_step=fused)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -735,6 +742,62 @@ def l2clip_run(steps, device, peaks):
             "fwd_gbs": round(bf / (ms_f * 1e-3) / 1e9, 1), "bwd_gbs": round(bb / (ms_b * 1e-3) / 1e9, 1),
             "fwd_frac_of_hbm": round(bf / (ms_f * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
             "bwd_frac_of_hbm": round(bb / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+
+
+def qclip_run(steps, device, peaks, w):
+    """The step of workload w with the L2Clip of q (learned scales, tau, threshold 9) fused
+    into the attention kernels (inkling_rel_attn_fwd_qclip / _bwd_qclip), against the same
+    step with the standalone L2Clip passes around the unfused attention; same inputs."""
+    from learned_relative_gqa_b200 import binding, workloads
+    x = workloads.make_inputs(w, device)
+    B, S, Hq, D = x["q"].shape
+    g = torch.Generator(device)
+    g.manual_seed(11)
+    xq = (x["q"].float() * (0.2 + 1.6 * torch.rand(B, S, Hq, 1, generator=g, device=device))).to(torch.bfloat16)
+    scale = 0.5 + torch.rand(Hq, D, generator=g, device=device)
+    tau = 0.5 + 1.5 * torch.rand(B, S, generator=g, device=device)
+    thr = 9.0
+    E = workloads.allowed_counts(w, x)
+    dims = binding.make_dims(xq, x["k"], x["profiles"], x["window"], x["query_offset"])
+    ldims = binding.make_l2clip_dims(xq, thr)
+    f32 = dict(dtype=torch.float32, device=device)
+    out, lse = torch.empty(xq.shape, **f32), torch.empty(xq.shape[:3], **f32)
+    qc = torch.empty_like(xq)
+    dx, dk, dv = torch.empty(xq.shape, **f32), torch.empty(x["k"].shape, **f32), torch.empty(x["v"].shape, **f32)
+    dprof, dsink = torch.empty(x["profiles"].shape, **f32), torch.empty(x["sink"].shape, **f32)
+    dscale, dtau, dq = torch.empty(Hq, D, **f32), torch.empty(B, S, **f32), torch.empty(xq.shape, **f32)
+    lib = binding.load()
+    ws = torch.empty(int(lib.inkling_rel_attn_qclip_workspace_size(ctypes.byref(dims), 1)), dtype=torch.uint8,
+                     device=device)
+    lws = torch.empty(binding.inkling_l2clip_workspace_size(ldims), dtype=torch.uint8, device=device)
+    a = (x["k"], x["v"], x["profiles"], x["sink"], x["valid"], x["key_valid"], x["positions"], x["key_positions"])
+    st = binding._stream(None)
+
+    def fused():
+        p = binding._p
+        binding._check(lib.inkling_rel_attn_fwd_qclip(
+            ctypes.byref(dims), thr, p(scale), p(tau), p(xq), *[p(t) for t in a[:4]], p(binding._u8(a[4])),
+            p(binding._u8(a[5])), p(a[6]), p(a[7]), p(qc), p(out), p(lse), p(ws), ws.numel(), st), "fwd_qclip")
+        binding._check(lib.inkling_rel_attn_bwd_qclip(
+            ctypes.byref(dims), thr, p(scale), p(tau), p(xq), p(qc), *[p(t) for t in a[:4]], p(binding._u8(a[4])),
+            p(binding._u8(a[5])), p(a[6]), p(a[7]), p(out), p(lse), p(x["dout"]), None, p(dx), p(dk), p(dv),
+            p(dprof), p(dsink), p(dscale), p(dtau), p(ws), ws.numel(), st), "bwd_qclip")
+
+    def separate():
+        binding.inkling_l2clip_fwd(ldims, xq, scale, tau, qc)
+        binding.inkling_rel_attn_fwd(dims, qc, *a, out, lse, ws)
+        binding.inkling_rel_attn_bwd(dims, qc, *a, out, lse, x["dout"], None, dq, dk, dv, dprof, dsink, ws)
+        binding.inkling_l2clip_bwd(ldims, xq, scale, tau, dq, dx, dscale, dtau, lws)
+
+    for _ in range(3):
+        fused()
+        separate()
+    ms_f = timed(fused, steps, torch.cuda.synchronize) / steps
+    ms_s = timed(separate, steps, torch.cuda.synchronize) / steps
+    fl = 14.0 * D * E
+    return {"workload": f"{w.name} S{w.seq} with the L2Clip of q (learned scales, tau, threshold 9), fwd+bwd",
+            "fused_ms": round(ms_f, 4), "separate_ms": round(ms_s, 4),
+            "fused_tflops": round(fl / (ms_f * 1e-3) / 1e12, 1), "separate_tflops": round(fl / (ms_s * 1e-3) / 1e12, 1)}
 
 
 def run_config(w, x, E, flops_step, world):

@@ -453,7 +453,9 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                         float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[cl]), __uint_as_float(sv[cl + 1])), sl2,
                                               make_float2(nl_c[u], nl_c[u + 1]));
                         if (USED) z = __ffma2_rn(make_float2(bias_c[u], bias_c[u + 1]), l2e, z);
-                        float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+                        float2 pr = ((IRA_DKDV_FMA_PAIRS >> ((cl >> 1) & 15)) & 1u)
+                                        ? exp2_fma2(z)
+                                        : make_float2(ex2_approx(z.x), ex2_approx(z.y));
                         bool ok0 = true, ok1 = true;
                         if (!PLAIN) {
                             ok0 = uint32_t(j - lo_c[u]) <= uint32_t(hi_c[u] - lo_c[u]) && cl < cl_lim;
@@ -908,6 +910,8 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
 
         issue_band(0);
         issue_band(1);
+        // the fused clip's epilogue reads this thread's part of its row of x: warm the L2
+        if (CLIP && row_in) prefetch_l2(p.q_raw + ((size_t(b) * p.S + i) * p.Hq + h) * D + w * (D / NWG));
         bool ok = true;
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 l2e = make_float2(kLog2e, kLog2e);
@@ -951,7 +955,8 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                     t = __ffma2_rn(make_float2(bf16hi_to_f32(v), bf16lo_to_f32(v)), l2e, nl2);
                 }
                 const float2 z = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t);
-                float2 pr = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+                float2 pr = ((IRA_DQ_FMA_PAIRS >> (pp & 15)) & 1u) ? exp2_fma2(z)
+                                                                   : make_float2(ex2_approx(z.x), ex2_approx(z.y));
                 if (need_mask) {
                     pr.x = (c >= c_lo && c <= c_hi) ? pr.x : 0.f;
                     pr.y = (c + 1 >= c_lo && c + 1 <= c_hi) ? pr.y : 0.f;

@@ -15,6 +15,19 @@ constexpr float kLn2 = 0.6931471805599453f;
 // more than this, so unnormalised probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f;
 
+// Which column pairs of a softmax thread's step take their exponentials on the FMA
+// pipe (bit u set: pair u of a 16-pair group, exp2_fma2) rather than the MUFU: the
+// forward, the dK/dV and the dQ kernels.
+#ifndef IRA_FWD_FMA_PAIRS
+#define IRA_FWD_FMA_PAIRS 0xAAAAu
+#endif
+#ifndef IRA_DKDV_FMA_PAIRS
+#define IRA_DKDV_FMA_PAIRS 0x0000u
+#endif
+#ifndef IRA_DQ_FMA_PAIRS
+#define IRA_DQ_FMA_PAIRS 0x0000u
+#endif
+
 // Default limit of every device-side wait (nanoseconds).
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 

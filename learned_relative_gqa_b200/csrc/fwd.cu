@@ -132,7 +132,8 @@ __device__ __forceinline__ void produce_ring(const CUtensorMap* tm, uint8_t* rin
 template <int D, int NH, bool CLIP>
 __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const int num_qtiles) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qc,
+               const AttnParams p, const int num_qtiles) {
     using L = Layout<D, NH>;
     constexpr int KB = L::KB;
     constexpr int K_WARP = 4 * NH, MMA_WARP = 4 * NH + 1, V_WARP = 4 * NH + 2, MMA_WARP_B = 4 * NH + 3;
@@ -293,6 +294,12 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     IRA_TRACE(p, 5 + s, n);
                 };
                 bool ok = mbar_wait(CLIP ? &q_ready[s] : q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
+                if (CLIP && ok) {
+                    // the clipped tile goes out to q_clipped by one tensor store (rows
+                    // beyond the sequence are not written); waited for before exit
+                    for (int kb = 0; kb < KB; ++kb) tma_store_4d(&tm_qc, q_smem(s, kb), kb * 64, h0 + s, i0, b);
+                    bulk_commit_group();
+                }
                 for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
                     ok = mbar_wait(&k_first[n], 0, ctl, p.err, kErrFwdK, p.timeout_ns);
                     if (!ok) break;
@@ -324,6 +331,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 // wait for every MMA of both issuers before TMEM is released
                 mma_commit(drain);
                 mbar_wait_drain(drain, 0);
+                if (CLIP) bulk_wait_all();
             }
         }
     } else {
@@ -396,9 +404,10 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
 
         if constexpr (CLIP) {
             // L2Clip of this row of q (head h): z = x * scale, y = z * min(1, thr / |z|) * tau,
-            // rounded to BF16, written over the Q tile in shared memory (for the products)
-            // and to q_clipped (for the backward). The tile is 128-byte swizzled: 16-byte
-            // chunk c of a row of a 64-column box sits at chunk c ^ (r mod 8) of that row.
+            // rounded to BF16 and written over the Q tile in shared memory, where the
+            // products read it and from where the MMA issuer stores the tile to q_clipped
+            // (for the backward). The tile is 128-byte swizzled: 16-byte chunk c of a row
+            // of a 64-column box sits at chunk c ^ (r mod 8) of that row.
             const bool q_ok = warp_wait(q_full, 0, ctl, p.err, kErrFwdQ, p.timeout_ns);
             const float* const sc = p.clip_scale ? p.clip_scale + size_t(h) * D : nullptr;
             auto chunk_at = [&](int c) {  // chunk c (8 columns) of the row
@@ -429,17 +438,15 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 const float nrm = sqrtf(ss);
                 float f = (nrm > p.clip_thr) ? p.clip_thr / nrm : 1.f;
                 if (p.clip_tau && row_in) f *= p.clip_tau[size_t(b) * p.S + i];
-                uint16_t* const grow = p.q_clipped + ((size_t(b) * p.S + i) * p.Hq + h) * D;
 #pragma unroll 1
                 for (int c = 0; c < D / 8; ++c) {
                     float z[8];
                     chunk_z(c, z);
-                    const uint4 y = make_uint4(pack_bf16x2(z[0] * f, z[1] * f), pack_bf16x2(z[2] * f, z[3] * f),
-                                               pack_bf16x2(z[4] * f, z[5] * f), pack_bf16x2(z[6] * f, z[7] * f));
-                    *reinterpret_cast<uint4*>(chunk_at(c)) = y;
-                    if (row_in) *reinterpret_cast<uint4*>(grow + 8 * c) = y;
+                    *reinterpret_cast<uint4*>(chunk_at(c)) =
+                        make_uint4(pack_bf16x2(z[0] * f, z[1] * f), pack_bf16x2(z[2] * f, z[3] * f),
+                                   pack_bf16x2(z[4] * f, z[5] * f), pack_bf16x2(z[6] * f, z[7] * f));
                 }
-                fence_proxy_async_smem();  // the tensor core reads these bytes next
+                fence_proxy_async_smem();  // the tensor core and the tensor store read these bytes next
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_ready[s]);
@@ -564,8 +571,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     const int c = 32 * q + 2 * u;
                     const float2 t =
                         __ffma2_rn(make_float2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), c2, nb2);
-                    // every second pair on the FMA pipe, the rest on the MUFU
-                    const float2 pr = (u & 1) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    // a share of the pairs on the FMA pipe, the rest on the MUFU
+                    const float2 pr = ((IRA_FWD_FMA_PAIRS >> u) & 1u) ? exp2_fma2(t)
+                                                                       : make_float2(ex2_approx(t.x), ex2_approx(t.y));
                     pk[u] = pack_bf16x2(pr.x, pr.y);
                     if (u & 1)
                         acc1 = __fadd2_rn(acc1, pr);
@@ -693,7 +701,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
 
 template <int D, int NH, bool CLIP>
 cudaError_t launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                        const AttnParams& p, cudaStream_t st) {
+                        const CUtensorMap& tm_qc, const AttnParams& p, cudaStream_t st) {
     using L = Layout<D, NH>;
     auto kern = fwd_kernel<D, NH, CLIP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
@@ -701,7 +709,7 @@ cudaError_t launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const 
     const int num_qtiles = (p.S + BM - 1) / BM;
     const long long grid = (long long)num_qtiles * p.B * (p.Hq / NH);
     if (grid == 0) return cudaSuccess;
-    kern<<<dim3(unsigned(grid)), dim3(32 * L::NWARPS), L::ALLOC, st>>>(tm_q, tm_k, tm_v, p, num_qtiles);
+    kern<<<dim3(unsigned(grid)), dim3(32 * L::NWARPS), L::ALLOC, st>>>(tm_q, tm_k, tm_v, tm_qc, p, num_qtiles);
     return cudaGetLastError();
 }
 
@@ -710,20 +718,23 @@ cudaError_t launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const 
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const AttnParams& p, cudaStream_t st) {
     const bool pair = (p.Hq / p.Hkv) % 2 == 0;
-    if (p.q_clipped) {
-        if (p.D == 128) {
-            return pair ? fwdk::launch_impl<128, 2, true>(tm_q, tm_k, tm_v, p, st)
-                        : fwdk::launch_impl<128, 1, true>(tm_q, tm_k, tm_v, p, st);
-        }
-        return pair ? fwdk::launch_impl<64, 2, true>(tm_q, tm_k, tm_v, p, st)
-                    : fwdk::launch_impl<64, 1, true>(tm_q, tm_k, tm_v, p, st);
-    }
     if (p.D == 128) {
-        return pair ? fwdk::launch_impl<128, 2, false>(tm_q, tm_k, tm_v, p, st)
-                    : fwdk::launch_impl<128, 1, false>(tm_q, tm_k, tm_v, p, st);
+        return pair ? fwdk::launch_impl<128, 2, false>(tm_q, tm_k, tm_v, tm_q, p, st)
+                    : fwdk::launch_impl<128, 1, false>(tm_q, tm_k, tm_v, tm_q, p, st);
     }
-    return pair ? fwdk::launch_impl<64, 2, false>(tm_q, tm_k, tm_v, p, st)
-                : fwdk::launch_impl<64, 1, false>(tm_q, tm_k, tm_v, p, st);
+    return pair ? fwdk::launch_impl<64, 2, false>(tm_q, tm_k, tm_v, tm_q, p, st)
+                : fwdk::launch_impl<64, 1, false>(tm_q, tm_k, tm_v, tm_q, p, st);
+}
+
+cudaError_t launch_fwd_qclip(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_qc, const AttnParams& p, cudaStream_t st) {
+    const bool pair = (p.Hq / p.Hkv) % 2 == 0;
+    if (p.D == 128) {
+        return pair ? fwdk::launch_impl<128, 2, true>(tm_q, tm_k, tm_v, tm_qc, p, st)
+                    : fwdk::launch_impl<128, 1, true>(tm_q, tm_k, tm_v, tm_qc, p, st);
+    }
+    return pair ? fwdk::launch_impl<64, 2, true>(tm_q, tm_k, tm_v, tm_qc, p, st)
+                : fwdk::launch_impl<64, 1, true>(tm_q, tm_k, tm_v, tm_qc, p, st);
 }
 
 }  // namespace ira

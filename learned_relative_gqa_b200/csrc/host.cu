@@ -566,13 +566,15 @@ inkling_status fwd_impl(const inkling_rel_attn_dims* dims, const uint16_t* q, co
     AttnParams p = base_params(dims, w, profiles, sink);
     p.out = out;
     p.lse = lse;
-    if (qc) {
-        p.clip_thr = qc->thr;
-        p.clip_scale = qc->scale;
-        p.clip_tau = qc->tau;
-        p.q_clipped = qc->q_clipped;
-    }
-    return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+    if (!qc) return cuda_status(tm.run([&] { return launch_fwd(tq, tk, tv, p, st); }));
+    p.clip_thr = qc->thr;
+    p.clip_scale = qc->scale;
+    p.clip_tau = qc->tau;
+    p.q_clipped = qc->q_clipped;
+    CUtensorMap tqc;
+    if (!encode_bhtd(&tqc, qc->q_clipped, dims->batch, dims->seq_q, dims->heads_q, dims->head_dim, 128))
+        return INKLING_ERR_CUDA;
+    return cuda_status(tm.run([&] { return launch_fwd_qclip(tq, tk, tv, tqc, p, st); }));
 }
 
 // The backward of either ABI; `qc` (optional) fuses the L2Clip backward of q in: q is

@@ -45,6 +45,10 @@ cudaError_t launch_l2clip_reduce(const float* dtau_part, int64_t T, int H, float
 // Forward attention. tm_q: {D, Hq, S, B} box {64,1,128,1}; tm_k / tm_v: {D, Hkv, Skv, B} box {64,1,64,1}.
 cudaError_t launch_fwd(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                        const AttnParams& p, cudaStream_t st);
+// The same with the L2Clip of q fused in (p.q_clipped set): tm_q maps the unclipped q,
+// tm_qc the clipped q it stores (same geometry).
+cudaError_t launch_fwd_qclip(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                             const CUtensorMap& tm_qc, const AttnParams& p, cudaStream_t st);
 
 // Backward attention. dkdv: tm_k / tm_v box {64,1,128,1}, tm_q / tm_do box {64,1,64,1},
 // tm_band: profiles as {R, B*Hq*S} with box {136, 8} (unused when R == 0).
