@@ -1013,14 +1013,23 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                     xv[8 * e8 + 2 * e + 1] = bf16hi_to_f32(wv[e]);
                 }
             }
+            // the learned scales of this warpgroup's columns (every lane reads the same
+            // addresses: broadcast accesses), four at a time
             const float* const scl = p.clip_scale ? p.clip_scale + size_t(h) * D + col : nullptr;
-            auto scv = [&](int e) { return scl ? scl[e] : 1.f; };
+            auto sc4 = [&](int e4) {
+                return scl ? *reinterpret_cast<const float4*>(scl + 4 * e4) : make_float4(1.f, 1.f, 1.f, 1.f);
+            };
             float zz = 0.f, zd = 0.f;
 #pragma unroll
-            for (int e = 0; e < DC; ++e) {
-                const float z = xv[e] * scv(e);
-                zz = fmaf(z, z, zz);
-                zd = fmaf(z, dy[e], zd);
+            for (int e4 = 0; e4 < DC / 4; ++e4) {
+                const float4 s = sc4(e4);
+                const float sv4[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float z = xv[4 * e4 + u] * sv4[u];
+                    zz = fmaf(z, z, zz);
+                    zd = fmaf(z, dy[4 * e4 + u], zd);
+                }
             }
             float2* const xrows = reinterpret_cast<float2*>(smem + L::XCH_OFF);
             float* const csum = reinterpret_cast<float*>(smem + L::XCH_OFF + 4 * NWG * 32 * 8);
@@ -1044,16 +1053,30 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             float* const stage = reinterpret_cast<float*>(smem + L::K_OFF) + (4 * w + wq) * 32 * STAGE_PITCH;
 #pragma unroll
-            for (int e = 0; e < DC; ++e) {  // dy becomes dx
-                const float dz = tau * c * (dy[e] - k2 * (xv[e] * scv(e)));
-                dy[e] = dz * scv(e);
-                stage[lane * STAGE_PITCH + e] = dz * xv[e];
+            for (int e4 = 0; e4 < DC / 4; ++e4) {  // dy becomes dx
+                const float4 s = sc4(e4);
+                const float sv4[4] = {s.x, s.y, s.z, s.w};
+                float dzx[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = 4 * e4 + u;
+                    const float dz = tau * c * (dy[e] - k2 * (xv[e] * sv4[u]));
+                    dy[e] = dz * sv4[u];
+                    dzx[u] = dz * xv[e];
+                }
+                *reinterpret_cast<float4*>(stage + lane * STAGE_PITCH + 4 * e4) = make_float4(dzx[0], dzx[1], dzx[2], dzx[3]);
             }
             __syncwarp();
             if (lane < DC) {
-                float a = 0.f;
-                for (int rr = 0; rr < 32; ++rr) a += stage[rr * STAGE_PITCH + lane];
-                csum[(w * 4 + wq) * 32 + lane] = a;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 32; rr += 4) {
+                    a0 += stage[rr * STAGE_PITCH + lane];
+                    a1 += stage[(rr + 1) * STAGE_PITCH + lane];
+                    a2 += stage[(rr + 2) * STAGE_PITCH + lane];
+                    a3 += stage[(rr + 3) * STAGE_PITCH + lane];
+                }
+                csum[(w * 4 + wq) * 32 + lane] = (a0 + a1) + (a2 + a3);
             }
             named_bar_sync(5 + w, 128);
             if (ok_out && wq == 0 && lane < DC) {

@@ -421,24 +421,29 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     z[2 * e] = bf16lo_to_f32(wv[e]);
                     z[2 * e + 1] = bf16hi_to_f32(wv[e]);
                 }
-                if (sc) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) z[e] *= sc[8 * c + e];
+                if (sc) {  // every lane reads the same 32 bytes: one broadcast access each
+                    const float4 s0 = *reinterpret_cast<const float4*>(sc + 8 * c);
+                    const float4 s1 = *reinterpret_cast<const float4*>(sc + 8 * c + 4);
+                    z[0] *= s0.x; z[1] *= s0.y; z[2] *= s0.z; z[3] *= s0.w;
+                    z[4] *= s1.x; z[5] *= s1.y; z[6] *= s1.z; z[7] *= s1.w;
                 }
             };
             if (q_ok) {
-                float ss = 0.f;
-#pragma unroll 1
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 4
                 for (int c = 0; c < D / 8; ++c) {
                     float z[8];
                     chunk_z(c, z);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(z[e], z[e], ss);
+                    for (int e = 0; e < 8; e += 2) {
+                        ss0 = fmaf(z[e], z[e], ss0);
+                        ss1 = fmaf(z[e + 1], z[e + 1], ss1);
+                    }
                 }
-                const float nrm = sqrtf(ss);
+                const float nrm = sqrtf(ss0 + ss1);
                 float f = (nrm > p.clip_thr) ? p.clip_thr / nrm : 1.f;
                 if (p.clip_tau && row_in) f *= p.clip_tau[size_t(b) * p.S + i];
-#pragma unroll 1
+#pragma unroll 4
                 for (int c = 0; c < D / 8; ++c) {
                     float z[8];
                     chunk_z(c, z);
