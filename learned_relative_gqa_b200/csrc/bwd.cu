@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 1, 0);
         mbar_init(kv_full, 1);
         // stage, score and accumulator barriers complete once both MMA issuers committed
         for (int u = 0; u < NST; ++u) {
@@ -177,6 +178,10 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     const int qt_first = tinfo[0];
     const int n_qt = (tinfo[1] >= tinfo[0]) ? tinfo[1] - tinfo[0] + 1 : 0;
     const int n_steps = n_qt * G;
+    if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 1, 1);
+        IRA_TRACE_GRID_INFO(p, 1, n_steps);
+    }
 
     auto k_smem = [&](int kb) { return smem + L::K_OFF + kb * KTILE; };
     auto v_smem = [&](int kb) { return smem + L::V_OFF + kb * KTILE; };
@@ -558,11 +563,13 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
         }
     }
 
+    if (threadIdx.x == 0) IRA_TRACE_GRID(p, 1, 4);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
+        if (lane == 0) IRA_TRACE_GRID(p, 1, 5);
     }
 }
 
@@ -683,6 +690,7 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 2, 0);
         mbar_init(q_full, 1);
         // a K stage is free once S (issuer A) and dQ (issuer B) of its step completed,
         // a V stage once dP (issuer B) did
@@ -731,6 +739,10 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
     const uint32_t tmem = *tmem_slot;
     const int t_begin = tinfo[0];
     const int n_steps = tinfo[1];
+    if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 2, 1);
+        IRA_TRACE_GRID_INFO(p, 2, n_steps);
+    }
 
     auto q_smem = [&](int kb) { return smem + L::Q_OFF + kb * QTILE; };
     auto do_smem = [&](int kb) { return smem + L::DO_OFF + kb * QTILE; };
@@ -883,26 +895,34 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
         const int m_r = (r + 1) & 7;
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
-        const size_t prof_at = trow * size_t(p.R);
-        const uint16_t* prof_row = (p.R > 0 && row_in && !empty) ? p.profiles + prof_at : nullptr;
         [[maybe_unused]] const long long prof_n = n_rows * p.R;
         // step n has distance offset delta = i0g - key0(n) = 64 (t_begin + n) - 64
         auto delta_of = [&](int n) { return BN * (t_begin + n) - BN; };
         // the warp's smallest distance in this warpgroup's columns is delta + 32 wq - cw - 15
         auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - cw - (COLS - 1) < p.R; };
-        // one cp.async group per call, also when nothing is copied
+        // The warp copies the windows of its 32 rows together: chunk k = 32 t + lane of its
+        // 32 x 3 chunks is chunk k mod 3 of row k / 3, so one copy instruction reads ~11
+        // contiguous row segments rather than 32 rows. One cp.async group per call, also
+        // when nothing is copied; a row is read only after every lane's wait and a
+        // __syncwarp.
+        const size_t prof_tile_at = ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R);
+        const uint16_t* const prof_tile = p.R > 0 ? p.profiles + prof_tile_at : nullptr;
         auto issue_band = [&](int n) {
             if (n < n_steps && band_needed(n)) {
-                const int x0 = delta_of(n) + r - cw - (COLS - 1) - m_r;
-                const uint32_t dst = smem_u32(band_wg + (n & 1) * BAND_BYTES) + uint32_t(unit) * 16u;
+                uint8_t* const dst_buf = band_wg + (n & 1) * BAND_BYTES;
+                const int dl = delta_of(n) - cw - (COLS - 1);
 #pragma unroll
-                for (int q = 0; q < BAND_CHUNKS; ++q) {
-                    const int d0 = x0 + 8 * q;
-                    const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
-                    const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                    if (IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, dst + 16u * q - smem_base, 16, L::TOTAL) &&
-                        IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, inb ? prof_at + d0 : 0, inb ? 8 : 0, prof_n))
-                        cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                for (int t = 0; t < BAND_CHUNKS; ++t) {
+                    const int k = 32 * t + lane;
+                    const int rr = wq * 32 + k / BAND_CHUNKS, q = k % BAND_CHUNKS;
+                    const int d0 = dl + rr - ((rr + 1) & 7) + 8 * q;
+                    const bool inb = prof_tile != nullptr && i0 + rr < p.S && d0 >= 0 && d0 < p.R;
+                    const size_t at = size_t(rr) * p.R + d0;
+                    const void* src = inb ? static_cast<const void*>(prof_tile + at) : p.safe_src;
+                    const uint32_t dst = smem_u32(dst_buf + band_unit(rr) * 16 + 16 * q);
+                    if (IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, dst - smem_base, 16, L::TOTAL) &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsDqGlobal, inb ? prof_tile_at + at : 0, inb ? 8 : 0, prof_n))
+                        cp_async_16(dst, src, inb ? 16u : 0u);
                 }
             }
             cp_async_commit();
@@ -934,14 +954,17 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
             tmem_ld16(tmem + lane_base + L::dp_col(bb) + cw, dp);
             uint32_t wv[COLS / 2 + 1];
             if (use_band) {
-                cp_async_wait_group<1>();  // this step's window (the next step's may fly)
+                cp_async_wait_group<1>();  // this step's windows (the next step's may fly)
+                __syncwarp();              // ... copied by every lane of the warp
                 const uint32_t* words = reinterpret_cast<const uint32_t*>(band_wg + (n & 1) * BAND_BYTES + unit * 16) + g_r;
                 const bool w_ok = IRA_IN_BOUNDS(p.err, kErrBoundsDqSmem, smem_u32(words) - smem_base,
                                                 4 * (COLS / 2 + 1), L::TOTAL);
 #pragma unroll
                 for (int q = 0; q < COLS / 2 + 1; ++q) wv[q] = w_ok ? words[q] : 0u;
             }
-            // this step's window is in registers: fetch the one of step n + 2 into its buffer
+            // this step's windows are in registers (every lane's: the copies are shared):
+            // fetch the ones of step n + 2 into their buffer
+            __syncwarp();
             issue_band(n + 2);
             tmem_wait_ld();
             const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
@@ -1167,11 +1190,13 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
         }
     }
 
+    if (threadIdx.x == 0) IRA_TRACE_GRID(p, 2, 4);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
+        if (lane == 0) IRA_TRACE_GRID(p, 2, 5);
     }
 }
 

@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     [[maybe_unused]] const long long n_rows = (long long)p.B * p.S * p.Hq;
 
     if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 0, 0);
         mbar_init(q_full, 1);
         // a K or V slot is free once the MMAs of every head's issuer have read it
         mbar_init(&k_first[0], 1);
@@ -224,6 +225,10 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     const uint32_t tmem = *tmem_slot;
     const int u_begin = tinfo[0];
     const int n_steps = tinfo[1];
+    if (threadIdx.x == 0) {
+        IRA_TRACE_GRID(p, 0, 1);
+        IRA_TRACE_GRID_INFO(p, 0, n_steps);
+    }
 
     auto q_smem = [&](int s, int kb) { return smem + L::Q_OFF + (s * KB + kb) * QBOX; };
     auto key0 = [&](int n) { return i0g + BN - (u_begin + n) * BN; };
@@ -365,43 +370,40 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         const int m_r = (r + 1) & 7;   // misalignment of the row's window start
         const int g_r = m_r >> 1;
         const uint32_t fshift = uint32_t(m_r & 1) * 16u;
-        const size_t prof_at = ((size_t(b) * p.Hq + h) * p.S + i) * size_t(p.R);
-        const uint16_t* prof_row = (p.R > 0 && row_in && !empty) ? p.profiles + prof_at : nullptr;
         [[maybe_unused]] const long long prof_n = (long long)p.B * p.Hq * p.S * p.R;
         auto delta_of = [&](int n) { return BN * (u_begin + n) - BN; };
         // the warp's smallest distance is delta + 32 wq - 63: no profile entry if >= R
         auto band_needed = [&](int n) { return delta_of(n) + wq * 32 - (BN - 1) < p.R; };
-        // copy this row's window of step n into band buffer (n & 1); always commits a
-        // group so that exactly two groups are outstanding at every wait below
+        // Copy the windows of step n of this warp's 32 rows into band buffer (n & 1). The
+        // warp copies its rows together: chunk k = 32 t + lane of the warp's 32 x 9 chunks
+        // is chunk k mod 9 of row k / 9, so the lanes of one copy instruction read a few
+        // contiguous row segments instead of 32 rows at once. Always commits a group, so
+        // that exactly two groups are outstanding at every wait below; a row is read only
+        // after every lane's wait and a __syncwarp.
+        const uint16_t* const prof_tile =
+            p.R > 0 ? p.profiles + ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) : nullptr;
         auto issue_band = [&](int n) {
             if (n < n_steps && band_needed(n)) {
-                const uint32_t dst = smem_u32(band0 + (n & 1) * BAND_BYTES + row_off);
-                const int x0 = delta_of(n) + r - (BN - 1) - m_r;
+                uint8_t* const dst_buf = band0 + (n & 1) * BAND_BYTES;
+                const int dl = delta_of(n);
 #pragma unroll
-                for (int q = 0; q < BAND_CHUNKS; ++q) {
-                    const int d0 = x0 + 8 * q;
-                    const bool inb = prof_row != nullptr && d0 >= 0 && d0 < p.R;
-                    const void* src = inb ? static_cast<const void*>(prof_row + d0) : p.safe_src;
-                    if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, dst + 16u * q - smem_base, 16, L::TOTAL) &&
-                        IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal, inb ? prof_at + d0 : 0, inb ? 8 : 0, prof_n))
-                        cp_async_16(dst + 16u * q, src, inb ? 16u : 0u);
+                for (int t = 0; t < BAND_CHUNKS; ++t) {
+                    const int k = 32 * t + lane;
+                    const int rr = wq * 32 + k / BAND_CHUNKS, q = k % BAND_CHUNKS;
+                    const int d0 = dl + rr - (BN - 1) - ((rr + 1) & 7) + 8 * q;
+                    const bool inb = prof_tile != nullptr && i0 + rr < p.S && d0 >= 0 && d0 < p.R;
+                    const size_t at = size_t(rr) * p.R + d0;
+                    const void* src = inb ? static_cast<const void*>(prof_tile + at) : p.safe_src;
+                    const uint32_t dst = smem_u32(dst_buf + band_slot(rr) * BAND_PITCH + 16 * q);
+                    if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, dst - smem_base, 16, L::TOTAL) &&
+                        IRA_IN_BOUNDS(p.err, kErrBoundsFwdGlobal,
+                                      inb ? ((size_t(b) * p.Hq + h) * p.S + i0) * size_t(p.R) + at : 0, inb ? 8 : 0,
+                                      prof_n))
+                        cp_async_16(dst, src, inb ? 16u : 0u);
                 }
             }
             cp_async_commit();
         };
-        // warm the L2 with the window of step n, well before its copy is issued
-        auto prefetch_band = [&](int n) {
-            if (n < n_steps && prof_row != nullptr) {
-                const int x0 = delta_of(n) + r - (BN - 1) - m_r;
-                if (x0 + 8 * BAND_CHUNKS > 0 && x0 < p.R) {
-                    const int lo = max(x0, 0), hi = min(x0 + 8 * BAND_CHUNKS, p.R) - 1;
-                    prefetch_l2(prof_row + lo);                    // the 144-byte window
-                    prefetch_l2(prof_row + min(lo + 64, hi));      // touches at most three
-                    prefetch_l2(prof_row + hi);                    // 128-byte lines
-                }
-            }
-        };
-
         if constexpr (CLIP) {
             // L2Clip of this row of q (head h): z = x * scale, y = z * min(1, thr / |z|) * tau,
             // rounded to BF16 and written over the Q tile in shared memory, where the
@@ -459,8 +461,6 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
 
         issue_band(0);
         issue_band(1);
-        prefetch_band(2);
-        prefetch_band(3);
         bool ok = true;
         for (int n = 0; n < n_steps; ++n) {
             const int buf = n & 1;
@@ -468,13 +468,13 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
             const bool my_full = empty || (rb.x <= jk && rb.y >= jk + BN - 1);
             const bool need_mask = !__all_sync(0xffffffffu, my_full);
             const bool use_band = band_needed(n);
-            prefetch_band(n + 4);
             if (!warp_wait(&s_full[2 * s + buf], (n >> 1) & 1, ctl, p.err, kErrFwdS, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             if (wq == 0 && lane == 0) IRA_TRACE(p, 11 + 3 * s, n);
             if (s == 0 && lane == 0) IRA_TRACE(p, 28 + wq, n);  // per-warp S ready (head A)
+            if (n == 0 && threadIdx.x == 0) IRA_TRACE_GRID(p, 0, 2);
             tc_fence_after();
             uint32_t x[64];
             tmem_ld32(tmem + lane_base + L::s_col(s, buf) + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -503,7 +503,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     constexpr bool BAND = decltype(band_c)::value, MASK = decltype(mask_c)::value;
                     uint32_t w[33];
                     if (BAND) {
-                        cp_async_wait_group<1>();  // this step's window (the next step's may fly)
+                        cp_async_wait_group<1>();  // this step's windows (the next step's may fly)
+                        __syncwarp();              // ... copied by every lane of the warp
                         if (s == 0 && lane == 0) IRA_TRACE(p, 24 + wq, n);  // per-warp band ready (head A)
                         const uint32_t* words =
                             reinterpret_cast<const uint32_t*>(band0 + buf * BAND_BYTES + row_off) + g_r;
@@ -545,7 +546,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 else mx = pass1(F_{}, T_{});
                 coef = kLog2e;
             }
-            // this step's band buffer is consumed: fetch the window of step n + 2 into it
+            // this step's band buffer is consumed (by every lane: the copies into it are
+            // shared): fetch the windows of step n + 2 into it
+            __syncwarp();
             issue_band(n + 2);
             if (wq == 0 && lane == 0) IRA_TRACE(p, 12 + 3 * s, n);
 
@@ -619,6 +622,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
             if (s == 0 && lane == 0) IRA_TRACE(p, 20 + wq, n);  // per-warp P done (head A)
         }
         cp_async_wait_all();
+        __syncwarp();  // the band rows, reused for staging below, are the warp's own
+        if (threadIdx.x == 0) IRA_TRACE_GRID(p, 0, 3);
 
         // ---- epilogue: O / l and lse ----
         if (ok && n_steps > 0) {
@@ -696,11 +701,13 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     }
 
     // ---- teardown ----
+    if (threadIdx.x == 0) IRA_TRACE_GRID(p, 0, 4);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
+        if (lane == 0) IRA_TRACE_GRID(p, 0, 5);
     }
 }
 

@@ -417,10 +417,34 @@ __device__ __forceinline__ void trace_event(unsigned long long* buf, int cta, in
     if (buf != nullptr && int(blockIdx.x) == cta && step < 8192) buf[step * 64 + ev] = clock64();
 }
 
+// Whole-grid record: slot (0..7) of this CTA's 8-word row in kernel kid's table
+// (8192 CTAs at most) after the step timeline receives the global timer
+// (nanoseconds), or `v` for trace_grid_value.
+__device__ __forceinline__ void trace_grid(unsigned long long* buf, int kid, int slot) {
+    if (buf != nullptr && blockIdx.x < 8192) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        buf[8192 * 64 + kid * 65536 + blockIdx.x * 8 + slot] = t;
+    }
+}
+__device__ __forceinline__ void trace_grid_value(unsigned long long* buf, int kid, int slot, unsigned long long v) {
+    if (buf != nullptr && blockIdx.x < 8192) buf[8192 * 64 + kid * 65536 + blockIdx.x * 8 + slot] = v;
+}
+__device__ __forceinline__ unsigned smid() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+
 }  // namespace ira
 
 #ifdef INKLING_TRACE
 #define IRA_TRACE(p, ev, step) ::ira::trace_event((p).trace, (p).trace_cta, (ev), (step))
+#define IRA_TRACE_GRID(p, kid, slot) ::ira::trace_grid((p).trace, (kid), (slot))
+#define IRA_TRACE_GRID_INFO(p, kid, n) \
+    ::ira::trace_grid_value((p).trace, (kid), 6, (unsigned long long)::ira::smid() | ((unsigned long long)(n) << 32))
 #else
 #define IRA_TRACE(p, ev, step) ((void)0)
+#define IRA_TRACE_GRID(p, kid, slot) ((void)0)
+#define IRA_TRACE_GRID_INFO(p, kid, n) ((void)0)
 #endif
