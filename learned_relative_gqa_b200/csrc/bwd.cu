@@ -786,7 +786,7 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                     else
                         tma_load_4d(k_smem(n, kb), &tm_k, &full[st], kb * 64, g, key0(n), b);
                 }
-                if (!is_v) IRA_TRACE(p, 41, n);
+                IRA_TRACE(p, is_v ? 50 : 41, n);
                 last = n;
             }
             if (!is_v) mbar_wait_drain(q_full, 0);
@@ -824,7 +824,7 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                 mma_commit(&s_full[bb]);
                 // last read of V(n) by B; A's read of K(n)
                 mma_commit(is_b ? &v_empty[n % NSV] : &k_empty[n % NSK]);
-                if (!is_b) IRA_TRACE(p, 42, n);
+                IRA_TRACE(p, is_b ? 51 : 42, n);
             };
             bool ok = mbar_wait(q_full, 0, ctl, p.err, kErrDqQ, p.timeout_ns);
             for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
@@ -962,11 +962,13 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
 #pragma unroll
                 for (int q = 0; q < COLS / 2 + 1; ++q) wv[q] = w_ok ? words[q] : 0u;
             }
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 52 + (w & 1), n);
             // this step's windows are in registers (every lane's: the copies are shared):
             // fetch the ones of step n + 2 into their buffer
             __syncwarp();
             issue_band(n + 2);
             tmem_wait_ld();
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 54 + (w & 1), n);
             const int c_lo = rb.x - jk, c_hi = rb.y - jk;  // allowed columns of this row
             uint32_t dk[COLS / 2];
 #pragma unroll
@@ -988,6 +990,7 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
                     __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nv2));
                 dk[pp] = pack_bf16x2(ds.x, ds.y);
             }
+            if (wq == 0 && lane == 0) IRA_TRACE(p, 56 + (w & 1), n);
             tmem_st8(tmem + lane_base + L::dp_col(bb) + cw, dk);
             tmem_wait_st();
             tc_fence_before();
