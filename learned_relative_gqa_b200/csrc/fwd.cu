@@ -54,9 +54,12 @@ namespace fwdk {
 
 constexpr int BM = 128;               // query rows per tile (TMEM lanes)
 constexpr int BN = 64;                // keys per step
-constexpr int KSLOTS = 3;             // K ring slots (two steps of lookahead)
-constexpr int VSLOTS = 2;             // V ring slots
-constexpr int NKV = 4;                // kv_ready barriers: step n's V(n) and K(n+2) on one barrier
+// K / V ring slots. A tile copy takes a few thousand cycles from issue to arrival while
+// the tensor core and L2 are busy, about a step and a half: K(n+2) is copied once S(n)
+// has read K(n) and is needed by S(n+2), issued after step n's probabilities; V(n+3) is
+// copied once PV(n) has read V(n) and is needed by PV(n+3), three steps of lead.
+constexpr int KSLOTS = 2;
+constexpr int VSLOTS = 3;
 constexpr int BAND_CHUNKS = 9;        // 16-byte chunks per band row (72 bf16)
 constexpr int BAND_PITCH = BAND_CHUNKS * 16;
 constexpr int BAND_BYTES = BM * BAND_PITCH;
@@ -77,9 +80,9 @@ struct Layout {
     static constexpr int V_OFF = K_OFF + KSLOTS * SLOT_BYTES;
     static constexpr int BAND_OFF = V_OFF + VSLOTS * SLOT_BYTES;
     static constexpr int BAR_OFF = BAND_OFF + NH * 2 * BAND_BYTES;
-    // q_full, k_first[2], kv_ready[NKV], k_empty[KSLOTS], v_empty[VSLOTS], drain,
+    // q_full, k_full[KSLOTS], v_full[VSLOTS], k_empty[KSLOTS], v_empty[VSLOTS], drain,
     // s_full[NH][2], p_full[NH][2], o_done[NH], o_full[NH], q_ready[NH]
-    static constexpr int NBARS = 4 + NKV + KSLOTS + VSLOTS + 7 * NH;
+    static constexpr int NBARS = 2 + 2 * (KSLOTS + VSLOTS) + 7 * NH;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 64;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -95,36 +98,26 @@ struct Layout {
 __device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return -floor_div(-a, b); }
 
-// Load K (or V) tiles 0 .. n_steps-1 of this CTA through a ring of NS slots
-// (lane 0 of the producer warp). V(n) and K(n+2) complete one barrier, kv_ready(n)
-// (two arrivals plus their bytes), so that the MMA issuers take a single wait per
-// step for the tiles of the step after; K(0) and K(1) have barriers of their own.
-// For the last two steps there is no K(n+2): the V producer then makes the second
-// arrival itself. Before returning, waits for its own copies in flight so that
-// none lands in the shared memory of an exiting CTA.
-template <int NS, int KB, bool IS_K>
-__device__ __forceinline__ void produce_ring(const CUtensorMap* tm, uint8_t* ring, uint64_t* k_first,
-                                             uint64_t* kv_ready, uint64_t* empty, int n_steps, int g, int b,
-                                             int key_first, CtaControl* ctl, const AttnParams& p, int site,
-                                             int trace_ev) {
-    // barrier and phase of load m
-    auto bar_of = [&](int m) { return IS_K ? (m < 2 ? &k_first[m] : &kv_ready[(m - 2) % NKV]) : &kv_ready[m % NKV]; };
-    auto phase_of = [&](int m) { return IS_K ? (m < 2 ? 0 : ((m - 2) / NKV) & 1) : (m / NKV) & 1; };
+// Load K (or V) tiles 0 .. n_steps-1 of this CTA through a ring of NS slots (lane 0 of
+// the producer warp): tile n goes to slot n mod NS once the MMAs of every head have
+// released it, and completes full[slot]. Before returning, waits for its own copies in
+// flight so that none lands in the shared memory of an exiting CTA.
+template <int NS, int KB>
+__device__ __forceinline__ void produce_ring(const CUtensorMap* tm, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                             int n_steps, int g, int b, int key_first, CtaControl* ctl,
+                                             const AttnParams& p, int site, int trace_ev) {
     int last = -1;
     for (int n = 0; n < n_steps; ++n) {
         const int slot = n % NS;
         if (!mbar_wait(&empty[slot], ((n / NS) & 1) ^ 1, ctl, p.err, site, p.timeout_ns)) break;
-        uint64_t* bar = bar_of(n);
-        if (!IS_K && n + 2 >= n_steps) mbar_arrive(bar);  // no K(n+2) exists
-        mbar_arrive_expect_tx(bar, KB * KBOX);
+        mbar_arrive_expect_tx(&full[slot], KB * KBOX);
         for (int kb = 0; kb < KB; ++kb)
             if (IRA_IN_BOUNDS(p.err, kErrBoundsFwdSmem, (slot * KB + kb) * KBOX, KBOX, NS * KB * KBOX))
-                tma_load_4d(ring + (slot * KB + kb) * KBOX, tm, bar, kb * 64, g, key_first - n * BN, b);
+                tma_load_4d(ring + (slot * KB + kb) * KBOX, tm, &full[slot], kb * 64, g, key_first - n * BN, b);
         IRA_TRACE(p, trace_ev, n);
         last = n;
     }
-    for (int n = (last >= NS ? last - NS + 1 : 0); n <= last; ++n)
-        mbar_wait_drain(bar_of(n), phase_of(n));
+    for (int n = (last >= NS ? last - NS + 1 : 0); n <= last; ++n) mbar_wait_drain(&full[n % NS], (n / NS) & 1);
 }
 
 // CLIP: the L2Clip of q is fused in (each softmax thread clips its row of the Q tile
@@ -144,9 +137,9 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_first = bars + 1;                   // [2]: K(0), K(1)
-    uint64_t* kv_ready = k_first + 2;               // [NKV]: V(n) and K(n+2)
-    uint64_t* k_empty = kv_ready + NKV;             // [KSLOTS]
+    uint64_t* k_full = bars + 1;                    // [KSLOTS]
+    uint64_t* v_full = k_full + KSLOTS;             // [VSLOTS]
+    uint64_t* k_empty = v_full + VSLOTS;            // [KSLOTS]
     uint64_t* v_empty = k_empty + KSLOTS;           // [VSLOTS]
     uint64_t* drain = v_empty + VSLOTS;
     uint64_t* s_full = drain + 1;                   // [NH][2]
@@ -179,9 +172,8 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
         IRA_TRACE_GRID(p, 0, 0);
         mbar_init(q_full, 1);
         // a K or V slot is free once the MMAs of every head's issuer have read it
-        mbar_init(&k_first[0], 1);
-        mbar_init(&k_first[1], 1);
-        for (int u = 0; u < NKV; ++u) mbar_init(&kv_ready[u], 2);  // the V and the K producer
+        for (int u = 0; u < KSLOTS; ++u) mbar_init(&k_full[u], 1);
+        for (int u = 0; u < VSLOTS; ++u) mbar_init(&v_full[u], 1);
         for (int u = 0; u < KSLOTS; ++u) mbar_init(&k_empty[u], NH);
         for (int u = 0; u < VSLOTS; ++u) mbar_init(&v_empty[u], NH);
         mbar_init(drain, NH);
@@ -247,7 +239,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 for (int s = 0; s < NH; ++s)
                     for (int kb = 0; kb < KB; ++kb)
                         tma_load_4d(q_smem(s, kb), &tm_q, q_full, kb * 64, h0 + s, i0, b);
-                produce_ring<KSLOTS, KB, true>(&tm_k, smem + L::K_OFF, k_first, kv_ready, k_empty, n_steps, g, b,
+                produce_ring<KSLOTS, KB>(&tm_k, smem + L::K_OFF, k_full, k_empty, n_steps, g, b,
                                                key0(0), ctl, p, kErrFwdKFree, 1);
                 mbar_wait_drain(q_full, 0);
             }
@@ -255,7 +247,7 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
             // -------------------------------------------------------- V producer
             if (lane == 0 && n_steps > 0) {
                 prefetch_tensormap(&tm_v);
-                produce_ring<VSLOTS, KB, false>(&tm_v, smem + L::V_OFF, k_first, kv_ready, v_empty, n_steps, g, b,
+                produce_ring<VSLOTS, KB>(&tm_v, smem + L::V_OFF, v_full, v_empty, n_steps, g, b,
                                                 key0(0), ctl, p, kErrFwdVFree, 2);
             }
         } else if (warp == MMA_WARP || (NH == 2 && warp == MMA_WARP_B)) {
@@ -271,9 +263,11 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                 constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
                 const uint32_t k_base = smem_u32(smem + L::K_OFF), v_base = smem_u32(smem + L::V_OFF);
                 const uint32_t q_base = smem_u32(q_smem(s, 0));
-                // V(n) and K(n+2) have landed (K(0) and K(1) have barriers of their own)
-                auto wait_kv = [&](int n) {
-                    return mbar_wait(&kv_ready[n % NKV], (n / NKV) & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
+                auto wait_k = [&](int n) {  // K(n) has landed
+                    return mbar_wait(&k_full[n % KSLOTS], (n / KSLOTS) & 1, ctl, p.err, kErrFwdK, p.timeout_ns);
+                };
+                auto wait_v = [&](int n) {  // V(n) has landed
+                    return mbar_wait(&v_full[n % VSLOTS], (n / VSLOTS) & 1, ctl, p.err, kErrFwdV, p.timeout_ns);
                 };
                 auto issue_s = [&](int n) {
                     const uint32_t kslot = k_base + (n % KSLOTS) * L::SLOT_BYTES;
@@ -306,30 +300,31 @@ __global__ void __launch_bounds__(32 * (4 * NH + 4), 1)
                     bulk_commit_group();
                 }
                 for (int n = 0; ok && n < 2 && n < n_steps; ++n) {
-                    ok = mbar_wait(&k_first[n], 0, ctl, p.err, kErrFwdK, p.timeout_ns);
+                    ok = wait_k(n);
                     if (!ok) break;
                     tc_fence_after();
                     issue_s(n);
                     mma_commit(&k_empty[n % KSLOTS]);
                 }
-                // The tiles of step n + 1 are awaited right after the MMAs of step n are
-                // queued, so that the path from P(n) to S(n+2) holds one wait only.
-                ok = ok && wait_kv(0);
                 for (int n = 0; ok && n < n_steps; ++n) {
                     // one barrier per S buffer: the softmax may already have finished
                     // step n + 1 (whose S was issued before this wait)
                     ok = mbar_wait(&p_full[2 * s + (n & 1)], (n >> 1) & 1, ctl, p.err, kErrFwdP, p.timeout_ns);
                     if (!ok) break;
                     IRA_TRACE(p, 7 + s, n);
+                    ok = wait_v(n);
+                    if (!ok) break;
+                    if (s == 0) IRA_TRACE(p, 10, n);
                     tc_fence_after();
                     issue_o(n);
                     mma_commit(&v_empty[n % VSLOTS]);
                     if (n + 2 < n_steps) {
+                        ok = wait_k(n + 2);
+                        if (!ok) break;
+                        tc_fence_after();
                         issue_s(n + 2);
                         mma_commit(&k_empty[(n + 2) % KSLOTS]);
                     }
-                    if (n + 1 < n_steps) ok = wait_kv(n + 1);
-                    if (s == 0) IRA_TRACE(p, 10, n + 1);
                 }
                 // O is final once every PV product has completed
                 if (ok) mma_commit(&o_full[s]);
