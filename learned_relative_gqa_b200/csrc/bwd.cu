@@ -6,7 +6,8 @@
 //   dq = scale sum_j dz k_j,  dk = scale sum_i dz q_i,  dv = sum_i P dout_i,
 //   dprofiles[b,h,i,d] = dz for the allowed key at distance d < R.
 // Dv, dsink, a BF16 copy of dout and lse*log2(e) come from the preprocessing
-// kernel; dprofiles entries that no allowed key reaches are zeroed there too.
+// kernel; dprofiles entries that no allowed key reaches are zeroed by a kernel of
+// their own.
 //
 // Two kernels, both tensor-core (tcgen05) with TMEM accumulators:
 //   * dkdv: one CTA per (batch, KV head, 128-key tile). It walks every query
@@ -18,9 +19,11 @@
 //     has exactly one allowed key.
 //   * dq: one CTA per (batch, query head, 128-row query tile) over 64-key
 //     tiles: S = Q K^T, dP = dO V^T, dQ += dS K (dS from TMEM). No atomics.
-// In both, S/dP are double buffered in TMEM and the two elementwise warpgroups
-// split the columns of every step (each owns half of them, with its own staged
-// profile rows), so the MMAs of step n+1 run while step n is being processed.
+// In both, four elementwise warpgroups split the columns of every step (16 each)
+// and S/dP sit in TMEM, double buffered in dkdv and in three buffers in dq, so the
+// MMAs of the next steps run while a step is being processed. dkdv's profile band
+// comes by TMA from a producer warp; in dq each warp copies its 32 rows' windows
+// for its warpgroup's columns.
 #include <cstddef>
 #include <type_traits>
 
@@ -887,9 +890,10 @@ __global__ void __launch_bounds__(32 * (4 * NWG + 4), 1)
         const float lse2 = row_in ? p.lse2t[trow] : 0.f;
         const float dvr = row_in ? p.dvt[trow] : 0.f;
 
-        // This thread's profile window for its columns, double buffered by step parity:
-        // column c = cw + cl of step n has distance delta(n) + r - c; the 16 columns'
-        // window starts (r + 1) mod 8 elements past a 16-byte boundary.
+        // This row's profile window for the warpgroup's columns (copied by the warp, see
+        // issue_band), double buffered by step parity: column c = cw + cl of step n has
+        // distance delta(n) + r - c; the 16 columns' window starts (r + 1) mod 8
+        // elements past a 16-byte boundary.
         const int unit = band_unit(r);
         uint8_t* const band_wg = smem + L::BAND_OFF + w * 2 * BAND_BYTES;
         const int m_r = (r + 1) & 7;

@@ -3,11 +3,11 @@
 // One CTA handles one 128-row query tile of NH query heads (NH = 2 heads of the
 // same KV group when the group size is even, else 1). Each step covers 64 keys;
 // its K and V tiles are loaded once by TMA and shared by both heads, K through a
-// three-slot ring and V through a two-slot ring, each fed by its own producer.
+// two-slot ring and V through a three-slot ring, each fed by its own producer.
 //
 //   warps 0..4*NH-1   softmax, one warpgroup per head (thread = query row =
-//                     TMEM lane); each thread also stages its own row's
-//                     profile window (double buffered, warmed in L2 ahead)
+//                     TMEM lane); each warp also stages its 32 rows' profile
+//                     windows (double buffered)
 //   warp  4*NH        TMA producer: Q (once), then the K tiles
 //   warp  4*NH+1      MMA issuer of head A (one thread): S = Q K^T (SMEM x SMEM
 //                     -> TMEM), O += P V (P from TMEM x V from SMEM -> TMEM)
@@ -34,9 +34,10 @@
 // [i_g0 + 64 - 64 u, i_g0 + 127 - 64 u], so its distance offset is
 // delta = 64 u - 64 and row r needs the distances [delta + r - 63, delta + r].
 // That window starts (r + 1) mod 8 elements past a 16-byte boundary for every
-// step; each softmax thread copies it (9 x 16 B, cp.async, zero fill outside
-// [0, R)) into a buffer whose rows are permuted so that the per-column 32-bit
-// reads of a warp hit 32 distinct shared-memory banks.
+// step; each warp copies the windows of its 32 rows (9 x 16 B each, cp.async, zero
+// fill outside [0, R); consecutive lanes take consecutive chunks of a row) into a
+// buffer whose rows are permuted so that the per-column 32-bit reads of a warp hit
+// 32 distinct shared-memory banks.
 //
 // Operation and argument conventions follow the NeMo AutoModel page for
 // Inkling2FlexAttention.forward; see include/inkling_rel_attn.h.
