@@ -112,3 +112,47 @@ def test_fused_qclip_equals_the_separate_passes():
                              x["positions"], x["key_positions"], **kw)
     torch.cuda.synchronize()
     assert float((out - o2).abs().max()) <= U.OUT_MAX and float((lse - l2).abs().max()) <= U.LSE_TOL
+
+
+def test_fused_qclip_full_size_matches_the_separate_passes():
+    """The training shape the bench times (B2 S8192 Hq32 Hkv4 D128, window 1024, R 1024,
+    documents), with learned scales, tau and threshold 9: the fused kernels against the
+    standalone L2Clip kernels around the unfused attention kernels (each checked against
+    its oracle in the tests above and in the attention parity tests), compared on the GPU
+    at the parity tolerances; the stored clipped q bit for bit except where the two FP32
+    evaluations round to neighbouring BF16 values."""
+    w = W.BY_NAME["train"]
+    x = W.make_inputs(w, "cuda", with_dout=True)
+    B, S, Hq, D = x["q"].shape
+    g = torch.Generator("cuda")
+    g.manual_seed(11)
+    xq = (x["q"].float() * (0.2 + 1.6 * torch.rand(B, S, Hq, 1, generator=g, device="cuda"))).to(torch.bfloat16)
+    scale = 0.5 + torch.rand(Hq, D, generator=g, device="cuda")
+    tau = 0.5 + 1.5 * torch.rand(B, S, generator=g, device="cuda")
+    a = (x["k"], x["v"], x["profiles"], x["sink"], x["valid"], x["key_valid"], x["positions"], x["key_positions"])
+    kw = dict(window=x["window"], query_offset=x["query_offset"])
+    out, lse, qc = binding.forward_qclip(xq, *a, threshold=9.0, clip_scale=scale, tau=tau, **kw)
+    gf = binding.backward_qclip(xq, qc, *a, out, lse, x["dout"], threshold=9.0, clip_scale=scale, tau=tau, **kw)
+    q2 = binding.l2clip_forward(xq, 9.0, scale, tau)
+    o2, l2 = binding.forward(q2, *a, **kw)
+    gs = binding.backward(q2, *a, o2, l2, x["dout"], **kw)
+    back = binding.l2clip_backward(xq, gs["dq"], 9.0, scale, tau)
+    torch.cuda.synchronize()
+
+    differ = (qc.view(torch.int16) != q2.view(torch.int16)).float().mean().item()
+    assert differ < 1e-3, f"{differ:.2e} of the clipped elements differ"
+
+    def close(a_, b_, tol, what, relative):
+        assert bool(torch.isfinite(a_).all()), f"{what}: non-finite values"
+        err = float((a_.double() - b_.double()).abs().max())
+        bound = tol * max(float(b_.abs().max()), 1e-30) if relative else tol
+        assert err <= bound, f"{what}: max abs err {err:.3e} > {bound:.3e}"
+
+    close(out, o2, U.OUT_MAX, "out", False)
+    assert float((out.double() - o2.double()).abs().mean()) <= U.OUT_MEAN
+    close(lse, l2, U.LSE_TOL, "lse", False)
+    for n_ in ("dk", "dv", "dprofiles", "dsink"):
+        close(gf[n_], gs[n_], U.GRAD_REL, n_, True)
+    close(gf["dx"], back["dx"], U.GRAD_REL, "dx", True)
+    close(gf["dclip_scale"], back["dscale"], U.GRAD_REL, "dclip_scale", True)
+    close(gf["dtau"], back["dtau"], U.GRAD_REL, "dtau", True)
