@@ -971,7 +971,10 @@ const char* inkling_rel_attn_last_cuda_error(void) {
 
 #ifdef INKLING_TRACE
 // Diagnostic builds only: record the pipeline timeline of CTA `cta` of the next
-// attention kernels into the device buffer `buf` (see ira::trace_event).
+// attention kernels (8192 steps x 64 events of 8 bytes, see ira::trace_event) and the
+// start / end stamps of every CTA of the forward, dK/dV and dQ kernels (three tables of
+// 8192 x 8 words after it, see ira::trace_grid) into the device buffer `buf`, which must
+// hold 8192 * 64 + 3 * 65536 words; `cta` = -1 records the CTA tables only.
 void inkling_rel_attn_debug_trace(void* buf, int cta) {
     g_trace_buf = static_cast<unsigned long long*>(buf);
     g_trace_cta = cta;
