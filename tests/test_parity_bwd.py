@@ -137,3 +137,13 @@ def test_forward_and_backward_replay_from_a_cuda_graph():
     assert torch.equal(out1, out0) and torch.equal(lse1, lse0)
     for n in NAMES:
         assert torch.equal(g1[n], g0[n]), n
+
+
+def test_backward_with_a_running_maximum_that_grows_every_step():
+    """The forward of test_forward_running_maximum_grows_every_step (O rescaled in every
+    step) feeding the backward: probabilities recomputed from its log-sum-exp."""
+    from tests.test_parity_fwd import ramp_profiles
+    w = U.custom("growing_max", 1, 320, 4, 2, 128, 0, 320, docs=(150, 300))
+    x = W.make_inputs(w, "cuda", with_dout=True)
+    ramp_profiles(x, 0.25)
+    check_full_bwd(x, with_dlse=True)

@@ -132,3 +132,23 @@ def test_forward_key_span_starts_and_ends_inside_words(seq_k):
     assert binding.inkling_rel_attn_validate(dims, x["valid"], x["key_valid"], x["positions"], x["key_positions"],
                                              ws) == binding.INKLING_OK
     check_full(x)
+
+
+def ramp_profiles(x, slope):
+    """profiles[b, h, i, d] = slope * d rounded to BF16 (the oracle reads the same values)."""
+    B, H, S, R = x["profiles"].shape
+    d = torch.arange(R, device=x["profiles"].device, dtype=torch.float32)
+    x["profiles"].copy_((slope * d).to(torch.bfloat16).expand(B, H, S, R))
+
+
+@pytest.mark.parametrize("slope", [0.25, 0.125])
+def test_forward_running_maximum_grows_every_step(slope):
+    """Profiles that rise with distance make each 64-key step's row maximum exceed the
+    running maximum by about 16 (slope 0.25) or 8 (slope 0.125) natural units, against a
+    lazy-rescale threshold of 8 log2 units = 5.5 natural units: the
+    steps visit keys from the diagonal outwards, so O is rescaled in every step after a
+    row's first (including the wait for the previous PV product)."""
+    w = U.custom("growing_max", 1, 320, 4, 2, 128, 0, 320, docs=(150, 300))
+    x = W.make_inputs(w, "cuda")
+    ramp_profiles(x, slope)
+    check_full(x)
