@@ -17,6 +17,8 @@ SMALL = [
     U.custom("window_one", 1, 300, 4, 2, 128, 1, 8),
     U.custom("extent_beyond_seq", 1, 192, 4, 4, 64, 0, 256, docs=(40, 100)),
     U.custom("group8_window", 1, 520, 8, 1, 128, 200, 200, docs=(60, 400)),
+    # no profiles, D 128, paired heads
+    U.custom("no_profiles_pairs", 2, 300, 8, 2, 128, 0, 0, docs=(30, 250), pad=(0, 20)),
 ]
 
 NAMES = ("dq", "dk", "dv", "dprofiles", "dsink")

@@ -19,6 +19,10 @@ SMALL = [
     U.custom("local_small", 1, 640, 8, 2, 128, 256, 256, pad=(0, 127)),
     U.custom("many_short_docs", 1, 384, 4, 2, 128, 0, 32, docs=(1, 7)),
     U.custom("d64_pairs_long", 1, 1000, 4, 2, 64, 0, 200, docs=(100, 700), pad=(0, 50)),
+    # no profiles, D 128, paired heads
+    U.custom("no_profiles_pairs", 2, 300, 8, 2, 128, 0, 0, docs=(30, 250), pad=(0, 20)),
+    U.custom("no_profiles_window_long", 1, 1100, 4, 2, 128, 200, 0, docs=(100, 900), pad=(0, 60)),
+    U.custom("no_profiles_offset_slice", 2, 160, 4, 1, 128, 0, 0, docs=(30, 150), seq_k=384, query_offset=200),
 ]
 
 
